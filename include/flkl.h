@@ -1,0 +1,151 @@
+/*
+ * flkl.h - C ABI of the fused linear-head + KL-divergence loss on B200 (sm_100a).
+ *
+ * The operation (the "Add FusedLinearKLDivLoss" pull-request page of the
+ * Liger-Kernel mirror, sections Summary and Details): given hidden states
+ * X[BT,H], a vocabulary head W[V,H] with optional bias b[V] and an explicit
+ * teacher distribution Q[BT,V],
+ *
+ *     z   = X W^T + b,   u = z / T,   log p = log_softmax(u) per row,
+ *     l_r = sum_v q_rv (log max(q_rv, eps) - log p_rv)   (q == 0 contributes 0)
+ *     loss = sum over kept rows of l_r / D
+ *
+ * with D = N_valid (batchmean), N_valid * V (mean) or 1 (sum); a row is dropped
+ * when its shift label equals ignore_index.  The gradients are produced in the
+ * same call ("gradient in forward", page Details, third bullet):
+ *
+ *     G_r = (S_r p_r - q_r) / (T D)  on kept rows, 0 on dropped rows,
+ *     S_r = sum_v q_rv,   dX = G W,   dW = G^T X,   db = sum_r G_r,
+ *
+ * and dW / db only when asked for (the frozen-head change of the GRPO page,
+ * section Summary).  The BT x V logits are never written to device memory: the
+ * library recomputes them tile by tile in two passes and stages only a
+ * bounded BT x Vc block of G (Vc <= V/8, rounded up to the tile width).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named "device" are CUDA device pointers on the current device;
+ *    the caller owns and allocates all of them (inputs, outputs, workspace).
+ *    The library allocates no device memory and keeps no per-call state.
+ *  - Tensors are dense and row-major.  Every tensor base pointer must be
+ *    16-byte aligned and H and V must be multiples of 8 (bf16) or 4 (fp32);
+ *    otherwise the call returns FLKL_ERR_UNSUPPORTED without launching.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t, may be NULL for the
+ *    legacy default stream).  A host-side argument error returns before any
+ *    launch.  A device-side error (a bounded wait that ran out) is recorded
+ *    in the workspace and read with flkl_device_status().
+ *  - No entry point throws, traps or aborts.
+ */
+#ifndef FLKL_H_
+#define FLKL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLKL_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define FLKL_API __attribute__((visibility("default")))
+#else
+#define FLKL_API
+#endif
+
+/* Reductions.  Same meaning as torch.nn.KLDivLoss, restricted to kept rows
+ * (page Details, first bullet).  FLKL_REDUCTION_NONE is refused with
+ * FLKL_ERR_UNSUPPORTED: the gradient is computed with the loss and needs a
+ * scalar loss (page Details, fourth bullet). */
+typedef enum {
+  FLKL_REDUCTION_BATCHMEAN = 0,
+  FLKL_REDUCTION_MEAN = 1,
+  FLKL_REDUCTION_SUM = 2,
+  FLKL_REDUCTION_NONE = 3
+} flkl_reduction;
+
+/* Element type shared by X, W, b and Q (and of dX). */
+typedef enum { FLKL_DTYPE_F32 = 0, FLKL_DTYPE_BF16 = 1 } flkl_dtype;
+
+typedef enum {
+  FLKL_OK = 0,
+  FLKL_ERR_INVALID_ARG = 1, /* null/inconsistent pointer, bad size or scalar */
+  FLKL_ERR_UNSUPPORTED = 2, /* reduction NONE, misalignment, size limits     */
+  FLKL_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed          */
+  FLKL_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out (kernel quit)  */
+  FLKL_ERR_WORKSPACE = 5    /* workspace missing, misaligned or too small    */
+} flkl_status;
+
+/* Version of this ABI (FLKL_ABI_VERSION of the built library). */
+FLKL_API int flkl_abi_version(void);
+
+/* Bytes of device workspace flkl_forward_backward needs for these sizes.
+ * Returns 0 for invalid sizes.  The workspace must be 256-byte aligned; its
+ * contents need no initialisation and are scratch between calls, except the
+ * status word read by flkl_device_status(). */
+FLKL_API size_t flkl_workspace_size(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW,
+                           int compute_db);
+
+/* Loss and gradients of the fused linear + KL(Q||P) loss, in one call.
+ *
+ *  X            device, [BT,H], dtype.
+ *  W            device, [V,H], dtype.
+ *  b            device, [V], dtype, or NULL (no bias).
+ *  Q            device, [BT,V], dtype: teacher probabilities, used as given
+ *               (not renormalised; rows need not sum to 1).
+ *  shift_labels device, [BT] int64, or NULL (every row kept).  Only equality
+ *               with ignore_index matters.
+ *  ignore_index label value that drops a row (usually -100).
+ *  BT, H, V     sizes; BT >= 0, H >= 1, V >= 1, each below 2^31.
+ *  dtype        flkl_dtype.  BF16 runs on the tensor cores with fp32
+ *               accumulation; F32 runs fp32 FMA throughout.
+ *  temperature  T > 0, divides the student logits only.
+ *  eps          >= 0; clamp inside log q only.
+ *  reduction    flkl_reduction.
+ *  compute_dW   nonzero: write dW; then dW must be non-NULL, else NULL.
+ *  compute_db   nonzero: write db; needs b and a non-NULL db, else db NULL.
+ *  accum_fp32   nonzero: dW and db are fp32; zero: they have `dtype`.
+ *  loss         device, one fp32 (written).
+ *  dX           device, [BT,H], dtype (overwritten).
+ *  dW           device, [V,H] (overwritten) or NULL.
+ *  db           device, [V] (overwritten) or NULL.
+ *  workspace    device, flkl_workspace_size(...) bytes, 256-byte aligned.
+ *  stream       cudaStream_t.
+ *
+ * Outputs are overwritten, never accumulated, and are gradients of the loss
+ * itself (an autograd wrapper multiplies them by the incoming gradient).
+ * Returns FLKL_OK once every kernel is enqueued.  With N_valid = 0 the loss
+ * and every gradient are 0.  BT = 0 writes loss 0 (and zero dW/db). */
+FLKL_API flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, const void* Q,
+                                  const int64_t* shift_labels, int64_t ignore_index, int64_t BT,
+                                  int64_t H, int64_t V, int dtype, float temperature, float eps,
+                                  int reduction, int compute_dW, int compute_db, int accum_fp32,
+                                  float* loss, void* dX, void* dW, void* db, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns the device status recorded by the last
+ * flkl_forward_backward call that used `workspace` (FLKL_OK or
+ * FLKL_ERR_TIMEOUT), or FLKL_ERR_CUDA if the copy or the synchronisation
+ * fails. */
+FLKL_API flkl_status flkl_device_status(const void* workspace, void* stream);
+
+/* Upper bound, in milliseconds, of every wait inside the kernels (default
+ * 4000).  After it a kernel records FLKL_ERR_TIMEOUT, drains its own copies,
+ * frees its tensor memory and returns.  Applies to later launches of this
+ * process; 0 restores the default. */
+FLKL_API void flkl_set_wait_limit_ms(unsigned int ms);
+
+/* Self-check of the bounded wait: launches one block that waits on an
+ * mbarrier which nothing ever completes, with a limit of `limit_ms`, and
+ * writes the resulting status code (FLKL_ERR_TIMEOUT expected) to the device
+ * int *status_out.  Touches no other memory. */
+FLKL_API flkl_status flkl_wait_selftest(int* status_out, unsigned int limit_ms, void* stream);
+
+/* Static text for a status code. */
+FLKL_API const char* flkl_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLKL_H_ */

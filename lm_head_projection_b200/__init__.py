@@ -1,0 +1,254 @@
+"""B200-native fused linear-head + KL-divergence loss (FusedLinearKLDivLoss).
+
+Python binding of the C ABI in ``include/flkl.h``.  It only marshals
+arguments: torch supplies device memory and the current stream, and every
+step of the computation runs in the CUDA library ``_flkl.so`` built from
+``csrc/`` (``python -m lm_head_projection_b200.build``).  There is no CPU or
+PyTorch fallback: without the built library every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "FLKL_OK", "FlklError", "flkl_abi_version", "flkl_workspace_size", "flkl_forward_backward",
+    "flkl_device_status", "flkl_set_wait_limit_ms", "flkl_wait_selftest", "flkl_status_string",
+    "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "_flkl.so")
+_LIB = None
+
+FLKL_OK = 0
+REDUCTIONS = {"batchmean": 0, "mean": 1, "sum": 2, "none": 3}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class FlklError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {flkl_status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {_LIB_PATH} is not built; run "
+                "`python -m lm_head_projection_b200.build` (nvcc, sm_100a)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        c = ctypes
+        lib.flkl_abi_version.restype = c.c_int
+        lib.flkl_abi_version.argtypes = []
+        lib.flkl_workspace_size.restype = c.c_size_t
+        lib.flkl_workspace_size.argtypes = [c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_int,
+                                            c.c_int]
+        lib.flkl_forward_backward.restype = c.c_int
+        lib.flkl_forward_backward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,      # X W b Q
+            c.c_void_p, c.c_int64,                               # labels ignore_index
+            c.c_int64, c.c_int64, c.c_int64, c.c_int,            # BT H V dtype
+            c.c_float, c.c_float, c.c_int,                       # T eps reduction
+            c.c_int, c.c_int, c.c_int,                           # dW db accum_fp32
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,      # loss dX dW db
+            c.c_void_p, c.c_size_t, c.c_void_p]                  # ws bytes stream
+        lib.flkl_device_status.restype = c.c_int
+        lib.flkl_device_status.argtypes = [c.c_void_p, c.c_void_p]
+        lib.flkl_set_wait_limit_ms.restype = None
+        lib.flkl_set_wait_limit_ms.argtypes = [c.c_uint]
+        lib.flkl_wait_selftest.restype = c.c_int
+        lib.flkl_wait_selftest.argtypes = [c.c_void_p, c.c_uint, c.c_void_p]
+        lib.flkl_status_string.restype = c.c_char_p
+        lib.flkl_status_string.argtypes = [c.c_int]
+        _LIB = lib
+    return _LIB
+
+
+# ------------------------------------------------------------------ raw C ABI
+
+def flkl_abi_version() -> int:
+    return _lib().flkl_abi_version()
+
+
+def flkl_status_string(status: int) -> str:
+    return _lib().flkl_status_string(int(status)).decode()
+
+
+def flkl_workspace_size(BT, H, V, dtype, compute_dW, compute_db) -> int:
+    return _lib().flkl_workspace_size(int(BT), int(H), int(V), int(dtype), int(bool(compute_dW)),
+                                      int(bool(compute_db)))
+
+
+def flkl_forward_backward(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype, temperature,
+                          eps, reduction, compute_dW, compute_db, accum_fp32, loss, dX, dW, db,
+                          workspace, workspace_bytes, stream) -> int:
+    """The C entry point with raw integer pointers (0 = NULL); returns the status."""
+    return _lib().flkl_forward_backward(
+        X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
+        int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
+        int(workspace_bytes), stream)
+
+
+def flkl_device_status(workspace_ptr, stream=None) -> int:
+    return _lib().flkl_device_status(workspace_ptr, stream)
+
+
+def flkl_set_wait_limit_ms(ms: int) -> None:
+    _lib().flkl_set_wait_limit_ms(int(ms))
+
+
+def flkl_wait_selftest(status_ptr, limit_ms, stream=None) -> int:
+    return _lib().flkl_wait_selftest(status_ptr, int(limit_ms), stream)
+
+
+# ------------------------------------------------------------------ torch-facing wrapper
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _check_dev(name, t, dtype, shape, device):
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor], Q: torch.Tensor,
+                     shift_labels: Optional[torch.Tensor] = None, ignore_index: int = -100,
+                     temperature: float = 1.0, eps: float = 1e-10, reduction: str = "batchmean",
+                     compute_dW: bool = True, compute_db: bool = False, accum_fp32: bool = True,
+                     out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None, check_status: bool = False) -> dict:
+    """Loss and gradients in one call on the current CUDA stream.
+
+    Allocates outputs (and the workspace) with torch unless given in ``out`` /
+    ``workspace``; returns ``{"loss", "dX", "dW", "db"}`` (None for the ones
+    not asked for).  Raises FlklError on a non-OK status.
+    """
+    if reduction not in REDUCTIONS:
+        raise ValueError(f"unknown reduction {reduction!r}")
+    if X.dtype not in DTYPES:
+        raise ValueError(f"dtype {X.dtype} not supported (float32 or bfloat16)")
+    dev = X.device
+    BT, H = X.shape
+    V = W.shape[0]
+    dt = X.dtype
+    _check_dev("X", X, dt, (BT, H), dev)
+    _check_dev("W", W, dt, (V, H), dev)
+    _check_dev("Q", Q, dt, (BT, V), dev)
+    if b is not None:
+        _check_dev("b", b, dt, (V,), dev)
+    if shift_labels is not None:
+        _check_dev("shift_labels", shift_labels, torch.int64, (BT,), dev)
+    compute_db = bool(compute_db and b is not None)
+    pdt = torch.float32 if (accum_fp32 or dt == torch.float32) else dt
+    out = {} if out is None else out
+    loss = out.get("loss")
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=dev)
+    dX = out.get("dX")
+    if dX is None:
+        dX = torch.empty_like(X)
+    dW = out.get("dW") if compute_dW else None
+    if compute_dW and dW is None:
+        dW = torch.empty((V, H), dtype=pdt, device=dev)
+    db = out.get("db") if compute_db else None
+    if compute_db and db is None:
+        db = torch.empty((V,), dtype=pdt, device=dev)
+    need = flkl_workspace_size(BT, H, V, DTYPES[dt], compute_dW, compute_db)
+    if need == 0:
+        raise FlklError(1, "flkl_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    status = flkl_forward_backward(
+        _ptr(X), _ptr(W), _ptr(b), _ptr(Q), _ptr(shift_labels), ignore_index, BT, H, V,
+        DTYPES[dt], temperature, eps, REDUCTIONS[reduction], compute_dW, compute_db, accum_fp32,
+        _ptr(loss), _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace), workspace.numel(),
+        st.cuda_stream)
+    if status != FLKL_OK:
+        raise FlklError(status, "flkl_forward_backward")
+    if check_status:
+        s = flkl_device_status(_ptr(workspace), st.cuda_stream)
+        if s != FLKL_OK:
+            raise FlklError(s, "flkl_forward_backward (device)")
+    return {"loss": loss, "dX": dX, "dW": dW, "db": db, "workspace": workspace}
+
+
+class _FusedLinearKLDivFunction(torch.autograd.Function):
+    """Gradient-in-forward: the forward call produces every gradient; the
+    backward only scales them by the incoming gradient of the loss."""
+
+    @staticmethod
+    def forward(ctx, X, W, b, Q, shift_labels, ignore_index, temperature, eps, reduction,
+                accum_fp32):
+        need_dW = ctx.needs_input_grad[1]
+        need_db = b is not None and ctx.needs_input_grad[2]
+        r = forward_backward(X.contiguous(), W.contiguous(),
+                             None if b is None else b.contiguous(), Q.contiguous(),
+                             shift_labels, ignore_index, temperature, eps, reduction,
+                             compute_dW=need_dW, compute_db=need_db, accum_fp32=accum_fp32)
+        ctx.save_for_backward(r["dX"], r["dW"], r["db"])
+        ctx.w_dtype = W.dtype
+        return r["loss"]
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        dX, dW, db = ctx.saved_tensors
+        one = bool((grad_out == 1).all())
+        if not one:
+            dX = dX * grad_out.to(dX.dtype)
+            dW = None if dW is None else dW * grad_out.to(dW.dtype)
+            db = None if db is None else db * grad_out.to(db.dtype)
+        if dW is not None:
+            dW = dW.to(ctx.w_dtype)
+        if db is not None:
+            db = db.to(ctx.w_dtype)
+        return dX, dW, db, None, None, None, None, None, None, None
+
+
+class FusedLinearKLDivLoss(torch.nn.Module):
+    """Module form with the options of the pull-request page (*Details*):
+    ``reduction`` ("batchmean" / "mean" / "sum"; "none" is refused),
+    ``ignore_index`` applied through ``shift_labels``, ``temperature``, ``eps``
+    and ``accum_dtype`` (torch.float32 keeps the head gradient in fp32).
+
+    ``forward(lin_weight, _input, target_probs, bias=None, shift_labels=None)``
+    """
+
+    def __init__(self, ignore_index: int = -100, reduction: str = "batchmean",
+                 temperature: float = 1.0, eps: float = 1e-10,
+                 accum_dtype: Optional[torch.dtype] = None):
+        super().__init__()
+        if reduction == "none":
+            raise ValueError("reduction='none' is not supported: the gradient is computed with "
+                             "the loss and needs a scalar loss; use an element-wise KL loss")
+        if reduction not in ("batchmean", "mean", "sum"):
+            raise ValueError(f"unknown reduction {reduction!r}")
+        self.ignore_index = ignore_index
+        self.reduction = reduction
+        self.temperature = temperature
+        self.eps = eps
+        self.accum_fp32 = accum_dtype == torch.float32
+
+    def forward(self, lin_weight, _input, target_probs, bias=None, shift_labels=None):
+        return _FusedLinearKLDivFunction.apply(_input, lin_weight, bias, target_probs,
+                                               shift_labels, self.ignore_index, self.temperature,
+                                               self.eps, self.reduction, self.accum_fp32)

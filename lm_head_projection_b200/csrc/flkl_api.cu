@@ -1,0 +1,440 @@
+// Host side of the C ABI declared in include/flkl.h: argument validation,
+// the pass plan and workspace layout, TMA tensor maps, and the launch
+// sequence on the caller's stream.
+//
+// Launch sequence of one call (bf16):
+//   k_prepare        N_valid, divisor D, 1/(T D); clears the status word
+//   pass 1  (tc)     z tiles = X W^T in TMEM, fused softmax/KL statistics
+//   k_combine        per-row lse and row loss, gradient coefficients
+//   k_loss           loss = sum of row losses / D (fixed order)
+//   per vocabulary chunk c of width Vc:
+//     pass 2 (tc)    z tiles of the chunk again, G = (S p - q)/(T D) -> bf16
+//                    staging [BT x Vc], db column partials
+//     dW gemm (tc)   dW[c] = G_c^T X (only when dW is asked for)
+//     dX gemm (tc)   dX (+)= G_c W[c] (fp32 partial across chunks)
+//   k_db_reduce      db (only when asked for)
+
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/flkl.h"
+#include "row_kernels.cuh"
+#include "simt_f32.cuh"
+#include "tc_gemm.cuh"
+
+namespace flkl {
+namespace {
+
+constexpr size_t kStagingBudget = size_t(256) << 20;  // bytes of G staging at most
+constexpr int kMaxDevices = 64;
+
+unsigned long long g_wait_limit_ns = 4000ull * 1000000ull;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+struct Plan {
+  bool tc;
+  int tile_m, tile_n;
+  long long m_tiles, n_tiles;  // pass tiles over [BT] x [V]
+  long long Vc, nchunks;
+  long long db_groups;
+  size_t off_st, off_rows, off_G, off_dx, off_db, total;
+};
+
+bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int compute_db,
+               Plan& p) {
+  (void)compute_dW;
+  if (BT < 0 || H < 1 || V < 1) return false;
+  if (BT >= (int64_t(1) << 31) || H >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return false;
+  if (dtype != FLKL_DTYPE_F32 && dtype != FLKL_DTYPE_BF16) return false;
+  p.tc = dtype == FLKL_DTYPE_BF16;
+  p.tile_m = p.tc ? TC_BM : ST_T;
+  p.tile_n = p.tc ? TC_BN : ST_T;
+  const size_t elem = p.tc ? 2 : 4;
+  p.m_tiles = cdiv(BT, p.tile_m);
+  p.n_tiles = cdiv(V, p.tile_n);
+  // Chunk width: at most V/8 (rounded up to the tile width) and at most the
+  // staging budget; never below one tile.
+  long long vc = cdiv(cdiv(V, 8), p.tile_n) * p.tile_n;
+  if (BT > 0) {
+    long long cap = static_cast<long long>(kStagingBudget / (size_t(BT) * elem));
+    cap = (cap / p.tile_n) * p.tile_n;
+    vc = std::min(vc, std::max<long long>(cap, p.tile_n));
+  }
+  vc = std::min(vc, p.n_tiles * p.tile_n);
+  p.Vc = vc;
+  p.nchunks = cdiv(V, vc);
+  p.db_groups = p.tc ? p.m_tiles * 4 : p.m_tiles;
+  size_t off = align256(sizeof(DevCtl));
+  p.off_st = off;
+  off += align256(size_t(5) * p.n_tiles * BT * 4);
+  p.off_rows = off;
+  off += align256(size_t(4) * BT * 4);
+  p.off_G = off;
+  off += align256(size_t(BT) * vc * elem);
+  p.off_dx = off;
+  if (p.nchunks > 1) off += align256(size_t(BT) * H * 4);
+  p.off_db = off;
+  if (compute_db) off += align256(size_t(p.db_groups) * V * 4);
+  p.total = off;
+  return true;
+}
+
+int g_num_sms[kMaxDevices] = {};
+std::mutex g_mu;
+
+int num_sms() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_num_sms[dev] = n > 0 ? n : 148;
+  }
+  return g_num_sms[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 2-D tensor map: extents {inner, outer}, row pitch in elements, box
+// {64, box_outer}, 128-byte swizzle, zero fill outside the extents.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+              uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <class Epi, bool A_MN, bool B_MN>
+cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& g,
+                      const typename Epi::Params& ep, cudaStream_t st) {
+  auto kern = tc_gemm_kernel<Epi, A_MN, B_MN>;
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = true;
+  }
+  const long long tiles = static_cast<long long>(g.m_tiles) * g.n_tiles;
+  if (tiles <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
+  kern<<<grid, TC_THREADS, TC_SMEM_BYTES, st>>>(ta, tb, g, ep);
+  return cudaGetLastError();
+}
+
+TcGemmArgs gemm_args(long long M, long long N, long long K, int m_fastest, int* err) {
+  TcGemmArgs g{};
+  g.M = static_cast<int>(M);
+  g.N = static_cast<int>(N);
+  g.K = static_cast<int>(K);
+  g.m_tiles = static_cast<int>(cdiv(M, TC_BM));
+  g.n_tiles = static_cast<int>(cdiv(N, TC_BN));
+  g.num_kb = static_cast<int>(cdiv(K, TC_BK));
+  g.m_fastest = m_fastest;
+  g.err_flag = err;
+  g.wait_limit_ns = g_wait_limit_ns;
+  return g;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define FLKL_CUDA(x)                               \
+  do {                                             \
+    if ((x) != cudaSuccess) return FLKL_ERR_CUDA;  \
+  } while (0)
+
+flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W,
+                   const __nv_bfloat16* b, const __nv_bfloat16* Q, const int64_t* labels,
+                   long long ignore_index, int BT, int H, int V, float T, float eps,
+                   int compute_dW, int compute_db, int accum_fp32, float* loss,
+                   __nv_bfloat16* dX, void* dW, void* db, uint8_t* ws, cudaStream_t st) {
+  DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
+  float* stats = reinterpret_cast<float*>(ws + P.off_st);
+  float* rows = reinterpret_cast<float*>(ws + P.off_rows);
+  float* lse2 = rows;
+  float* coefS = rows + BT;
+  float* coefQ = rows + 2 * static_cast<size_t>(BT);
+  float* rowloss = rows + 3 * static_cast<size_t>(BT);
+  __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(ws + P.off_G);
+  float* dxpart = reinterpret_cast<float*>(ws + P.off_dx);
+  float* dbpart = compute_db ? reinterpret_cast<float*>(ws + P.off_db) : nullptr;
+  int* err = &ctl->err;
+  const float LOG2E = 1.4426950408889634f;
+  const float t_scale = LOG2E / T;
+
+  CUtensorMap mX_k, mW_k, mX_mn, mW_mn;
+  if (!make_map(&mX_k, X, H, BT, H, TC_BM) || !make_map(&mW_k, W, H, V, H, TC_BN) ||
+      !make_map(&mX_mn, X, H, BT, H, 64) || !make_map(&mW_mn, W, H, V, H, 64))
+    return FLKL_ERR_CUDA;
+
+  // pass 1: statistics over all V
+  {
+    TcGemmArgs g = gemm_args(BT, V, H, 1, err);
+    EpiStats::Params ep{Q, b, BT, V, t_scale, eps, stats,
+                        static_cast<long long>(P.n_tiles) * BT};
+    FLKL_CUDA((launch_tc<EpiStats, false, false>(mX_k, mW_k, g, ep, st)));
+  }
+  k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
+      stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+      coefQ, rowloss);
+  FLKL_CUDA(cudaGetLastError());
+  k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
+  FLKL_CUDA(cudaGetLastError());
+
+  const int ldg = static_cast<int>(P.Vc);
+  for (long long c = 0; c < P.nchunks; ++c) {
+    const int c0 = static_cast<int>(c * P.Vc);
+    const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
+    // pass 2: gradient of the chunk's logits -> bf16 staging
+    {
+      TcGemmArgs g = gemm_args(BT, Vw, H, 1, err);
+      g.b_n_off = c0;
+      EpiGrad::Params ep{Q, b, BT, V, c0, ldg, G, t_scale, lse2, coefS, coefQ, dbpart};
+      FLKL_CUDA((launch_tc<EpiGrad, false, false>(mX_k, mW_k, g, ep, st)));
+    }
+    CUtensorMap mG_k, mG_mn;
+    if (!make_map(&mG_k, G, Vw, BT, ldg, TC_BM) || !make_map(&mG_mn, G, Vw, BT, ldg, 64))
+      return FLKL_ERR_CUDA;
+    if (compute_dW) {
+      TcGemmArgs g = gemm_args(Vw, H, BT, 0, err);
+      EpiStoreRows::Params ep{dW, H, Vw, H, c0, accum_fp32};
+      FLKL_CUDA((launch_tc<EpiStoreRows, true, true>(mG_mn, mX_mn, g, ep, st)));
+    }
+    {
+      TcGemmArgs g = gemm_args(BT, H, Vw, 0, err);
+      g.b_k_off = c0;
+      int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
+      EpiAccumRows::Params ep{dxpart, dX, H, BT, H, mode};
+      FLKL_CUDA((launch_tc<EpiAccumRows, false, true>(mG_k, mW_mn, g, ep, st)));
+    }
+  }
+  if (compute_db) {
+    k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
+        dbpart, static_cast<int>(P.db_groups), V, db, accum_fp32);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  return FLKL_OK;
+}
+
+flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* b, const float* Q,
+                    const int64_t* labels, long long ignore_index, int BT, int H, int V, float T,
+                    float eps, int compute_dW, int compute_db, float* loss, float* dX, float* dW,
+                    float* db, uint8_t* ws, cudaStream_t st) {
+  DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
+  float* stats = reinterpret_cast<float*>(ws + P.off_st);
+  float* rows = reinterpret_cast<float*>(ws + P.off_rows);
+  float* lse2 = rows;
+  float* coefS = rows + BT;
+  float* coefQ = rows + 2 * static_cast<size_t>(BT);
+  float* rowloss = rows + 3 * static_cast<size_t>(BT);
+  float* G = reinterpret_cast<float*>(ws + P.off_G);
+  float* dxpart = reinterpret_cast<float*>(ws + P.off_dx);
+  float* dbpart = compute_db ? reinterpret_cast<float*>(ws + P.off_db) : nullptr;
+  const float t_scale = 1.4426950408889634f / T;
+  const unsigned mt = static_cast<unsigned>(P.m_tiles);
+
+  k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
+      X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT);
+  FLKL_CUDA(cudaGetLastError());
+  k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
+      stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+      coefQ, rowloss);
+  FLKL_CUDA(cudaGetLastError());
+  k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
+  FLKL_CUDA(cudaGetLastError());
+
+  const int ldg = static_cast<int>(P.Vc);
+  for (long long c = 0; c < P.nchunks; ++c) {
+    const int c0 = static_cast<int>(c * P.Vc);
+    const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
+    k_simt_grad<<<dim3(static_cast<unsigned>(cdiv(Vw, ST_T)), mt), 256, 0, st>>>(
+        X, W, b, Q, BT, H, V, c0, Vw, t_scale, lse2, coefS, coefQ, G, ldg, dbpart);
+    FLKL_CUDA(cudaGetLastError());
+    if (compute_dW) {
+      // dW[c0 + v][h] = sum_r G[r][v] X[r][h]
+      k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)),
+                             static_cast<unsigned>(cdiv(Vw, ST_T))),
+                        256, 0, st>>>(G, 1, ldg, X, 1, H, Vw, H, BT, nullptr, dW, H, c0, 4);
+      FLKL_CUDA(cudaGetLastError());
+    }
+    const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
+    // dX[r][h] (+)= sum_v G[r][v] W[c0 + v][h]
+    k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)), mt), 256, 0, st>>>(
+        G, ldg, 1, W + static_cast<size_t>(c0) * H, 1, H, BT, H, Vw, dxpart, dX, H, 0, mode);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  if (compute_db) {
+    k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
+        dbpart, static_cast<int>(P.db_groups), V, db, 1);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  return FLKL_OK;
+}
+
+__global__ void k_wait_selftest(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    *status = 0;
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl wc{&abort_flag, status, limit_ns};
+    // Nothing arrives on `bar`: the wait must run out and record the status.
+    (void)mbar_wait(&bar, 0, wc);
+  }
+}
+
+}  // namespace
+}  // namespace flkl
+
+using namespace flkl;
+
+extern "C" {
+
+int flkl_abi_version(void) { return FLKL_ABI_VERSION; }
+
+size_t flkl_workspace_size(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW,
+                           int compute_db) {
+  Plan p;
+  if (!make_plan(BT, H, V, dtype, compute_dW, compute_db, p)) return 0;
+  return p.total;
+}
+
+void flkl_set_wait_limit_ms(unsigned int ms) {
+  g_wait_limit_ns = (ms == 0 ? 4000ull : static_cast<unsigned long long>(ms)) * 1000000ull;
+}
+
+const char* flkl_status_string(int s) {
+  switch (s) {
+    case FLKL_OK: return "ok";
+    case FLKL_ERR_INVALID_ARG: return "invalid argument";
+    case FLKL_ERR_UNSUPPORTED: return "unsupported argument (reduction none, alignment or size)";
+    case FLKL_ERR_CUDA: return "CUDA runtime error";
+    case FLKL_ERR_TIMEOUT: return "a device-side wait ran out of time";
+    case FLKL_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, const void* Q,
+                                  const int64_t* shift_labels, int64_t ignore_index, int64_t BT,
+                                  int64_t H, int64_t V, int dtype, float temperature, float eps,
+                                  int reduction, int compute_dW, int compute_db, int accum_fp32,
+                                  float* loss, void* dX, void* dW, void* db, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  // ---- scalar arguments
+  if (dtype != FLKL_DTYPE_F32 && dtype != FLKL_DTYPE_BF16) return FLKL_ERR_INVALID_ARG;
+  if (reduction == FLKL_REDUCTION_NONE) return FLKL_ERR_UNSUPPORTED;
+  if (reduction < FLKL_REDUCTION_BATCHMEAN || reduction > FLKL_REDUCTION_SUM)
+    return FLKL_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !(temperature < INFINITY)) return FLKL_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(eps < INFINITY)) return FLKL_ERR_INVALID_ARG;
+  if (BT < 0 || H < 1 || V < 1) return FLKL_ERR_INVALID_ARG;
+  if (BT >= (int64_t(1) << 31) || H >= (int64_t(1) << 31) || V >= (int64_t(1) << 31))
+    return FLKL_ERR_UNSUPPORTED;
+  const int vec = dtype == FLKL_DTYPE_BF16 ? 8 : 4;
+  if (H % vec != 0 || V % vec != 0) return FLKL_ERR_UNSUPPORTED;
+  // ---- pointers
+  if (W == nullptr || loss == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (BT > 0 && (X == nullptr || Q == nullptr || dX == nullptr)) return FLKL_ERR_INVALID_ARG;
+  if ((compute_dW != 0) != (dW != nullptr)) return FLKL_ERR_INVALID_ARG;
+  if ((compute_db != 0) != (db != nullptr)) return FLKL_ERR_INVALID_ARG;
+  if (compute_db && b == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(b) || !aligned16(Q) || !aligned16(dX) ||
+      !aligned16(dW) || !aligned16(db) || (reinterpret_cast<uintptr_t>(shift_labels) & 7u) ||
+      (reinterpret_cast<uintptr_t>(loss) & 3u))
+    return FLKL_ERR_UNSUPPORTED;
+  Plan P;
+  if (!make_plan(BT, H, V, dtype, compute_dW, compute_db, P)) return FLKL_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < P.total)
+    return FLKL_ERR_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int bt = static_cast<int>(BT), h = static_cast<int>(H), v = static_cast<int>(V);
+
+  k_prepare<<<1, 1024, 0, st>>>(shift_labels, bt, static_cast<long long>(ignore_index), reduction,
+                                v, temperature, reinterpret_cast<DevCtl*>(ws));
+  FLKL_CUDA(cudaGetLastError());
+
+  if (BT == 0) {
+    // No rows: loss 0, and zero parameter gradients when asked for.
+    k_zero<<<1, 32, 0, st>>>(loss, sizeof(float));
+    FLKL_CUDA(cudaGetLastError());
+    const size_t pe = (dtype == FLKL_DTYPE_F32 || accum_fp32) ? 4 : 2;
+    if (compute_dW) {
+      const size_t bytes = size_t(V) * H * pe;
+      k_zero<<<static_cast<unsigned>(cdiv(bytes, 16 * 256)), 256, 0, st>>>(dW, bytes);
+      FLKL_CUDA(cudaGetLastError());
+    }
+    if (compute_db) {
+      const size_t bytes = size_t(V) * pe;
+      k_zero<<<static_cast<unsigned>(cdiv(bytes, 16 * 256)), 256, 0, st>>>(db, bytes);
+      FLKL_CUDA(cudaGetLastError());
+    }
+    return FLKL_OK;
+  }
+
+  if (P.tc) {
+    return run_tc(P, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
+                  static_cast<const __nv_bfloat16*>(b), static_cast<const __nv_bfloat16*>(Q),
+                  shift_labels, ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db,
+                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st);
+  }
+  return run_f32(P, static_cast<const float*>(X), static_cast<const float*>(W),
+                 static_cast<const float*>(b), static_cast<const float*>(Q), shift_labels,
+                 ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db, loss,
+                 static_cast<float*>(dX), static_cast<float*>(dW), static_cast<float*>(db), ws,
+                 st);
+}
+
+flkl_status flkl_device_status(const void* workspace, void* stream) {
+  if (workspace == nullptr) return FLKL_ERR_WORKSPACE;
+  int h = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FLKL_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FLKL_ERR_CUDA;
+  return h == 0 ? FLKL_OK : static_cast<flkl_status>(h);
+}
+
+flkl_status flkl_wait_selftest(int* status_out, unsigned int limit_ms, void* stream) {
+  if (status_out == nullptr) return FLKL_ERR_INVALID_ARG;
+  k_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      status_out, static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  return cudaGetLastError() == cudaSuccess ? FLKL_OK : FLKL_ERR_CUDA;
+}
+
+}  // extern "C"

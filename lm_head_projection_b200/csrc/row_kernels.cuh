@@ -1,0 +1,147 @@
+// Small SIMT kernels around the GEMMs: valid-row count and divisor, merge of
+// the per-tile softmax/KL statistics into per-row log-sum-exp and row loss,
+// the deterministic loss sum, and the db column reduction.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace flkl {
+
+// Device-side control block at the start of the workspace.
+struct DevCtl {
+  int err;       // first device error code of the call (0 = none)
+  int n_valid;   // rows whose shift label differs from ignore_index
+  float D;       // reduction divisor
+  float scale;   // 1 / (T * D), 0 when no row is kept
+  float invD;    // 1 / D, 0 when no row is kept
+};
+
+// One block of 1024 threads.  Counts kept rows (a row is dropped when its
+// shift label equals ignore_index), derives the divisor of the reduction
+// (batchmean: N_valid, mean: N_valid * V, sum: 1) and resets the error flag.
+__global__ void __launch_bounds__(1024) k_prepare(const int64_t* __restrict__ labels, int BT,
+                                                  long long ignore_index, int reduction, int V,
+                                                  float temperature, DevCtl* ctl) {
+  __shared__ int warp_cnt[32];
+  int cnt = 0;
+  if (labels == nullptr) {
+    cnt = (threadIdx.x == 0) ? BT : 0;
+  } else {
+    for (int i = threadIdx.x; i < BT; i += blockDim.x) cnt += (labels[i] != ignore_index) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) n += warp_cnt[w];
+    float D = 1.f;
+    if (reduction == 0) D = static_cast<float>(n);
+    else if (reduction == 1) D = static_cast<float>(n) * static_cast<float>(V);
+    ctl->err = 0;
+    ctl->n_valid = n;
+    ctl->D = D;
+    ctl->scale = n > 0 ? 1.f / (temperature * D) : 0.f;
+    ctl->invD = n > 0 ? 1.f / D : 0.f;
+  }
+}
+
+// Merge of the per-tile statistics (m, s, A, B2, S) of each row, in tile
+// order, into lse2 = log2 sum 2^t and the row loss
+//   l_r = ln2 * B2 - A / T + ln2 * lse2 * S
+// (= sum_v q (log max(q,eps) - log p)).  Also the per-row coefficients of the
+// gradient pass.  Block: 8 warps x 32 rows; warp w merges tiles w, w+8, ...
+__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ st, int n_tiles, int BT,
+                                                 const int64_t* __restrict__ labels,
+                                                 long long ignore_index, float invT,
+                                                 const DevCtl* __restrict__ ctl,
+                                                 float* __restrict__ lse2_out,
+                                                 float* __restrict__ coefS,
+                                                 float* __restrict__ coefQ,
+                                                 float* __restrict__ rowloss) {
+  __shared__ float part[8][5][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * 32 + lane;
+  const size_t plane = static_cast<size_t>(n_tiles) * BT;
+  float m = -INFINITY, s = 0.f, A = 0.f, B2 = 0.f, S = 0.f;
+  if (row < BT) {
+    for (int t = w; t < n_tiles; t += 8) {
+      const size_t o = static_cast<size_t>(t) * BT + row;
+      const float tm = st[o], ts = st[o + plane];
+      const float nm = fmaxf(m, tm);
+      s = s * exp2f(m - nm) + ts * exp2f(tm - nm);
+      m = nm;
+      A += st[o + 2 * plane];
+      B2 += st[o + 3 * plane];
+      S += st[o + 4 * plane];
+    }
+  }
+  part[w][0][lane] = m;
+  part[w][1][lane] = s;
+  part[w][2][lane] = A;
+  part[w][3][lane] = B2;
+  part[w][4][lane] = S;
+  __syncthreads();
+  if (w == 0 && row < BT) {
+    m = part[0][0][lane];
+    s = part[0][1][lane];
+    A = part[0][2][lane];
+    B2 = part[0][3][lane];
+    S = part[0][4][lane];
+    for (int k = 1; k < 8; ++k) {
+      const float tm = part[k][0][lane];
+      if (tm == -INFINITY) continue;  // warp k saw no tile of this row
+      const float nm = fmaxf(m, tm);
+      s = s * exp2f(m - nm) + part[k][1][lane] * exp2f(tm - nm);
+      m = nm;
+      A += part[k][2][lane];
+      B2 += part[k][3][lane];
+      S += part[k][4][lane];
+    }
+    const float LN2 = 0.693147180559945309f;
+    const float lse2 = m + log2f(s);
+    const bool keep = labels == nullptr || labels[row] != ignore_index;
+    const float sc = ctl->scale;
+    lse2_out[row] = lse2;
+    coefS[row] = keep ? S * sc : 0.f;
+    coefQ[row] = keep ? sc : 0.f;
+    rowloss[row] = keep ? (LN2 * B2 - A * invT + LN2 * lse2 * S) : 0.f;
+  }
+}
+
+// loss = (sum of row losses) / D, summed in a fixed order (fp64 partials).
+__global__ void __launch_bounds__(1024) k_loss(const float* __restrict__ rowloss, int BT,
+                                               const DevCtl* __restrict__ ctl, float* loss) {
+  __shared__ double red[1024];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < BT; i += blockDim.x) acc += static_cast<double>(rowloss[i]);
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (static_cast<int>(threadIdx.x) < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *loss = static_cast<float>(red[0] * static_cast<double>(ctl->invD));
+}
+
+// db[v] = sum over row groups g (in order) of part[g][v].
+__global__ void k_db_reduce(const float* __restrict__ part, int groups, int V, void* db,
+                            int out_fp32) {
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v >= V) return;
+  float acc = 0.f;
+  for (int gi = 0; gi < groups; ++gi) acc += part[static_cast<size_t>(gi) * V + v];
+  if (out_fp32) static_cast<float*>(db)[v] = acc;
+  else static_cast<__nv_bfloat16*>(db)[v] = __float2bfloat16_rn(acc);
+}
+
+// Zero fill (used for empty inputs).
+__global__ void k_zero(void* p, size_t bytes) {
+  const size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 16;
+  if (i + 16 <= bytes) *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p) + i) = make_uint4(0, 0, 0, 0);
+  else
+    for (size_t j = i; j < bytes; ++j) static_cast<uint8_t*>(p)[j] = 0;
+}
+
+}  // namespace flkl

@@ -1,0 +1,132 @@
+"""C-ABI boundary tests that need no GPU: the library loads, exports every
+symbol the header declares, sizes its workspace without any BT x V term, and
+rejects bad arguments on the host before launching anything.
+
+The argument-rejection tests pass placeholder pointer values that must never
+reach a kernel, so they only run where no GPU is visible.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import lm_head_projection_b200 as pkg
+from lm_head_projection_b200.workloads import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flkl.h")
+
+OK, INVALID, UNSUPPORTED, CUDA, TIMEOUT, WORKSPACE = range(6)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"FLKL_API\s+[\w\s\*]*?\b(flkl_\w+)\s*\(", text)
+
+
+def test_library_exports_every_declared_symbol():
+    syms = declared_symbols()
+    assert len(syms) >= 7
+    lib = ctypes.CDLL(pkg.library_path())
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_abi_version_and_status_strings():
+    assert pkg.flkl_abi_version() == 1
+    for s in range(6):
+        assert pkg.flkl_status_string(s)
+    assert "unknown" in pkg.flkl_status_string(99)
+
+
+def test_workspace_size_rules():
+    ws = pkg.flkl_workspace_size
+    assert ws(-1, 64, 64, 1, 1, 0) == 0
+    assert ws(4, 0, 64, 1, 1, 0) == 0
+    assert ws(4, 64, 0, 1, 1, 0) == 0
+    assert ws(4, 64, 64, 7, 1, 0) == 0
+    assert ws(0, 64, 64, 1, 1, 0) > 0
+    assert ws(4, 64, 64, 1, 1, 1) > ws(4, 64, 64, 1, 1, 0)
+    assert ws(4, 64, 64, 1, 1, 0) % 256 == 0
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_workspace_has_no_bt_by_v_buffer(name):
+    """The staged gradient block is at most BT x V/8 (plus tile rounding), and
+    the logits are never stored: the whole workspace stays well below one
+    BT x V array of the input dtype."""
+    w = WORKLOADS[name]
+    elem = 4 if w.dtype == "fp32" else 2
+    need = pkg.flkl_workspace_size(w.BT, w.H, w.V, 0 if w.dtype == "fp32" else 1, w.compute_dW,
+                                   w.compute_db)
+    full = w.BT * w.V * elem
+    if w.V >= 8 * 256:
+        assert need < 0.35 * full, (need, full)
+
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(),
+                            reason="placeholder pointers must not reach a real device")
+
+P = 4096  # placeholder, 16-byte aligned, never dereferenced
+
+
+def call(**kw):
+    a = dict(X=P, W=P, b=None, Q=P, shift_labels=None, ignore_index=-100, BT=64, H=64, V=64,
+             dtype=1, temperature=1.0, eps=1e-10, reduction=0, compute_dW=1, compute_db=0,
+             accum_fp32=1, loss=P, dX=P, dW=P, db=None, workspace=P, workspace_bytes=0,
+             stream=None)
+    a.update(kw)
+    return pkg.flkl_forward_backward(**a)
+
+
+@no_gpu
+@pytest.mark.parametrize("kw,expect", [
+    (dict(reduction=3), UNSUPPORTED),           # reduction none refused
+    (dict(reduction=7), INVALID),
+    (dict(dtype=5), INVALID),
+    (dict(temperature=0.0), INVALID),
+    (dict(temperature=-1.0), INVALID),
+    (dict(temperature=float("nan")), INVALID),
+    (dict(temperature=float("inf")), INVALID),
+    (dict(eps=-1e-3), INVALID),
+    (dict(eps=float("nan")), INVALID),
+    (dict(BT=-1), INVALID),
+    (dict(H=0), INVALID),
+    (dict(V=0), INVALID),
+    (dict(H=60), UNSUPPORTED),                  # bf16 rows must be 16-byte multiples
+    (dict(V=1004), UNSUPPORTED),
+    (dict(dtype=0, H=62), UNSUPPORTED),
+    (dict(BT=1 << 31), UNSUPPORTED),
+    (dict(W=None), INVALID),
+    (dict(X=None), INVALID),
+    (dict(Q=None), INVALID),
+    (dict(loss=None), INVALID),
+    (dict(dX=None), INVALID),
+    (dict(dW=None), INVALID),                   # compute_dW without dW
+    (dict(compute_dW=0), INVALID),              # dW given while frozen
+    (dict(compute_db=1, db=P), INVALID),        # db without bias
+    (dict(compute_db=1, b=P), INVALID),         # db pointer missing
+    (dict(compute_db=0, b=P, db=P), INVALID),   # db given but not asked for
+    (dict(X=P + 8), UNSUPPORTED),               # misaligned
+    (dict(Q=P + 4), UNSUPPORTED),
+    (dict(dX=P + 2), UNSUPPORTED),
+    (dict(shift_labels=P + 4), UNSUPPORTED),
+    (dict(workspace=None), WORKSPACE),
+    (dict(workspace=P + 16, workspace_bytes=1 << 40), WORKSPACE),  # not 256-aligned
+    (dict(workspace_bytes=100), WORKSPACE),     # too small
+])
+def test_host_rejects_bad_arguments(kw, expect):
+    assert call(**kw) == expect
+
+
+@no_gpu
+def test_empty_rows_allow_null_row_tensors_but_need_workspace():
+    assert call(BT=0, X=None, Q=None, dX=None, workspace_bytes=0) == WORKSPACE
+
+
+def test_python_module_refuses_reduction_none():
+    with pytest.raises(ValueError):
+        pkg.FusedLinearKLDivLoss(reduction="none")
