@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Throughput of the fused linear-head + KL-divergence loss (forward + backward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one flkl_forward_backward call over one batch of BT rows: loss, dX
+and (when the workload trains the head) dW/db, with every input resident in
+device memory.  Prints one JSON line on rank 0.
+
+* value      rows (tokens) per second over all ranks, timed with CUDA events
+             on the launch stream around exactly K steps (max over ranks);
+* e2e        the same metric through the public Python API with the batch
+             (X, Q, labels) copied from pinned host memory every step and the
+             loss read back to the host every step; the head W stays resident;
+* roofline   the dominant kernel (largest share of the step's device time)
+             from a second, profiled run of K steps: its GEMM FLOPs per launch
+             over its average launch time, against the measured bf16 peak;
+* cpu_baseline  the fp64 oracle on the host cores on a bounded row sample.
+
+Multi-GPU (launched with torch.distributed.run): every rank runs its own
+batch (weak scaling, data parallel); the only collectives are the timing
+barrier and the max-over-ranks reduction of the elapsed time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from lm_head_projection_b200.workloads import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "fwd+bwd tokens/s at H=4096,V=128256 bf16; % of roofline (tensor/HBM)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_KINDS = {"stats", "grad", "dW", "dX"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample-rows", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="flkl_clocks_", suffix=".csv")
+        self.proc = None
+        self.t_start = time.time()
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[3], parts[4:]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        # samples under load: the upper half of the observed clocks
+        clocks = sorted(r[0] for r in rows)
+        active = [r for r in rows if r[0] >= clocks[len(clocks) // 4]]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3][1:5])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in active), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} needs {n_gpus} ranks (WORLD_SIZE={world}); launch "
+                         "with python -m torch.distributed.run --nproc-per-node N")
+    return world, rank, local
+
+
+def oracle_sample(w, rows, seed=123):
+    """Inputs of a `rows`-row sample of workload `w` (fresh draw), as fp64
+    numpy arrays, plus the oracle's keyword arguments."""
+    import numpy as np
+
+    inp = make_inputs(w.with_(BT=rows, seed=seed), device="cpu")
+    f = lambda t: None if t is None else t.float().numpy().astype(np.float64)
+    args = (f(inp["X"]), f(inp["W"]), f(inp["b"]), f(inp["Q"]))
+    kw = dict(shift_labels=None if inp["shift_labels"] is None else inp["shift_labels"].numpy(),
+              ignore_index=inp["ignore_index"], temperature=inp["temperature"], eps=inp["eps"],
+              reduction=inp["reduction"], compute_dW=inp["compute_dW"],
+              compute_db=inp["compute_db"])
+    return args, kw
+
+
+def host_threads():
+    cores = len(os.sched_getaffinity(0))
+    try:
+        from threadpoolctl import threadpool_info
+        nt = max((i.get("num_threads", 0) for i in threadpool_info()), default=0)
+        cores = nt or cores
+    except Exception:
+        pass
+    return cores
+
+
+def time_oracle(args, kw):
+    from oracle import forward_backward as oracle_fb
+
+    t0 = time.perf_counter()
+    oracle_fb(*args, **kw)
+    return time.perf_counter() - t0
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch.distributed as dist
+
+    import lm_head_projection_b200 as pkg
+
+    world, rank, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    w = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    inp = make_inputs(w, device=dev)
+    X, W, b, Q, lab = inp["X"], inp["W"], inp["b"], inp["Q"], inp["shift_labels"]
+    dt_code = pkg.DTYPES[X.dtype]
+    compute_db = inp["compute_db"]
+    r0 = pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
+                              inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
+                              compute_db=compute_db, accum_fp32=inp["accum_fp32"],
+                              check_status=True)
+    ws = r0["workspace"]
+    out = {k: r0[k] for k in ("loss", "dX", "dW", "db")}
+    stream = torch.cuda.current_stream(dev)
+    p = lambda t: None if t is None else t.data_ptr()
+    call_args = (p(X), p(W), p(b), p(Q), p(lab), inp["ignore_index"], w.BT, w.H, w.V, dt_code,
+                 inp["temperature"], inp["eps"], pkg.REDUCTIONS[inp["reduction"]],
+                 inp["compute_dW"], compute_db, inp["accum_fp32"], p(out["loss"]), p(out["dX"]),
+                 p(out["dW"]), p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
+
+    def step():
+        s = pkg.flkl_forward_backward(*call_args)
+        if s != 0:
+            raise pkg.FlklError(s, "flkl_forward_backward")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local
+    clocks = ClockSampler(gpu_index)
+    time.sleep(0.3)
+
+    # ---------------- timed region: exactly K steps
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = pkg.flkl_device_status(ws.data_ptr(), stream.cuda_stream)
+    if status != 0:
+        raise pkg.FlklError(status, "device status after the timed region")
+
+    # ---------------- per-launch breakdown: K profiled steps
+    cap = 256
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+    for e in events:  # torch creates the CUDA event on its first record
+        e.record(stream)
+    torch.cuda.synchronize()
+    per_kind = {}
+    launches_per_step = 0
+    kernel_flops = {}
+    for _ in range(args.steps):
+        st, kinds, n = pkg.flkl_forward_backward_profiled(*call_args, events, cap)
+        if st != 0:
+            raise pkg.FlklError(st, "flkl_forward_backward_profiled")
+        launches_per_step = n
+        torch.cuda.synchronize()
+        for i, k in enumerate(kinds):
+            name = pkg.LAUNCH_KINDS[k]
+            d = per_kind.setdefault(name, [0.0, 0])
+            d[0] += events[2 * i].elapsed_time(events[2 * i + 1])
+            d[1] += 1
+    clocks.stop()
+    clk = clocks.summary()
+
+    # GEMM FLOPs per step of each kind (2*M*N*K summed over its launches)
+    base = 2.0 * w.BT * w.H * w.V
+    kernel_flops = {"stats": base, "grad": base, "dX": base,
+                    "dW": base if inp["compute_dW"] else 0.0}
+    total_prof_ms = sum(v[0] for v in per_kind.values())
+    dominant = max(per_kind, key=lambda k: per_kind[k][0])
+    peaks, peaks_src = load_peaks()
+    peak_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    dom_ms, dom_n = per_kind[dominant]
+    if dominant in GEMM_KINDS:
+        launches_of_kind_per_step = dom_n / args.steps
+        flops_per_launch = kernel_flops[dominant] / launches_of_kind_per_step
+        achieved = flops_per_launch / (dom_ms / dom_n * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_sust,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4), "traffic": None,
+                    "kernel": f"tc_gemm_kernel<{dominant}>",
+                    "peak_note": f"bf16_tflops_sustained of {peaks_src}",
+                    "share": round(dom_ms / total_prof_ms, 3)}
+    else:
+        roofline = {"bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": None, "traffic": None, "kernel": dominant}
+    breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step":
+                     round(v[1] / args.steps, 2), "share": round(v[0] / total_prof_ms, 3)}
+                 for k, v in sorted(per_kind.items())}
+
+    ms_per_step = ms / args.steps
+    tokens = w.BT * world
+    value = tokens / (ms_per_step * 1e-3)
+    counted = w.flops_counted()
+    step_tflops = counted / (ms_per_step * 1e-3) / 1e12
+    roof_time = max(counted / (peaks["bf16_tflops"] * 1e12),
+                    (algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9)))
+    step_roofline = {"counted_flops": counted, "tflops": round(step_tflops, 1),
+                     "frac_of_burst": round(roof_time / (ms_per_step * 1e-3), 4),
+                     "frac_of_sustained": round(
+                         max(counted / (peak_sust * 1e12),
+                             algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9))
+                         / (ms_per_step * 1e-3), 4),
+                     "peaks": peaks_src}
+
+    # ---------------- end to end: batch from pinned host memory, loss back
+    hX = X.cpu().pin_memory()
+    hQ = Q.cpu().pin_memory()
+    hL = None if lab is None else lab.cpu().pin_memory()
+    hloss = torch.empty((), dtype=torch.float32).pin_memory()
+    h2d = hX.numel() * hX.element_size() + hQ.numel() * hQ.element_size() + \
+        (0 if hL is None else hL.numel() * 8)
+    for _ in range(max(1, args.warmup)):
+        X.copy_(hX, non_blocking=True)
+        Q.copy_(hQ, non_blocking=True)
+        pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
+                             inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
+                             compute_db=compute_db, accum_fp32=inp["accum_fp32"], out=out,
+                             workspace=ws)
+        hloss.copy_(out["loss"], non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        X.copy_(hX, non_blocking=True)
+        Q.copy_(hQ, non_blocking=True)
+        if hL is not None:
+            lab.copy_(hL, non_blocking=True)
+        pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
+                             inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
+                             compute_db=compute_db, accum_fp32=inp["accum_fp32"], out=out,
+                             workspace=ws)
+        hloss.copy_(out["loss"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(tokens / (e2e_ms / args.steps * 1e-3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = min(args.cpu_sample_rows, w.BT)
+        oa, okw = oracle_sample(w, rows)
+        dt = time_oracle(oa, okw)
+        cores = host_threads()
+        cpu = {"value": round(rows / dt, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} rows of {w.name} (full H, V, same flags), fp64 numpy, "
+                         f"inputs pre-converted to fp64, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.BT * world, "BT_per_gpu": w.BT,
+                       "H": w.H, "V": w.V, "compute_dW": w.compute_dW,
+                       "compute_db": bool(compute_db), "reduction": w.reduction,
+                       "temperature": w.temperature, "parallelism": f"dp{world}",
+                       "l2": "inputs larger than L2 (W, Q), no flush"},
+            "e2e": e2e, "roofline": roofline, "step_roofline": step_roofline,
+            "kernels": breakdown, "gpu_launches": int(launches_per_step * args.steps),
+            "clocks": clk, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def algorithmic_bytes(w) -> float:
+    """X, W, Q and labels read once, dX and dW/db written once."""
+    e = 4 if w.dtype == "fp32" else 2
+    pe = 4 if (w.accum_fp32 or w.dtype == "fp32") else 2
+    b = w.BT * w.H * e * 2 + w.V * w.H * e + w.BT * w.V * e
+    if w.compute_dW:
+        b += w.V * w.H * pe
+    if w.bias:
+        b += w.V * e + (w.V * pe if w.compute_db else 0)
+    if w.ignore_frac > 0:
+        b += w.BT * 8
+    return float(b)
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    rows = max(1, min(args.ref_rows, w.BT))
+    oa, okw = oracle_sample(w, rows)
+    for _ in range(args.warmup):
+        time_oracle(oa, okw)
+    times = [time_oracle(oa, okw) for _ in range(args.steps)]
+    cores = host_threads()
+    total = sum(times)
+    value = rows * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": rows, "H": w.H, "V": w.V,
+                   "parallelism": "host"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"{rows} rows of {w.name} per step (full H, V, same "
+                                   "flags), fp64 numpy oracle, inputs pre-converted to fp64"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

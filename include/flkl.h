@@ -123,6 +123,34 @@ FLKL_API flkl_status flkl_forward_backward(const void* X, const void* W, const v
                                   float* loss, void* dX, void* dW, void* db, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* Kinds of launches reported by flkl_forward_backward_profiled. */
+typedef enum {
+  FLKL_LAUNCH_PREPARE = 0,  /* valid-row count and divisor                   */
+  FLKL_LAUNCH_STATS = 1,    /* pass 1: logits GEMM + softmax/KL statistics    */
+  FLKL_LAUNCH_COMBINE = 2,  /* per-row log-sum-exp and row loss              */
+  FLKL_LAUNCH_LOSS = 3,     /* reduction of the row losses                   */
+  FLKL_LAUNCH_GRAD = 4,     /* pass 2: logits GEMM again + G to staging      */
+  FLKL_LAUNCH_DW = 5,       /* dW chunk GEMM                                 */
+  FLKL_LAUNCH_DX = 6,       /* dX chunk GEMM                                 */
+  FLKL_LAUNCH_DB = 7,       /* db column reduction                           */
+  FLKL_LAUNCH_ZERO = 8      /* zero fill (BT = 0)                            */
+} flkl_launch_kind;
+
+/* flkl_forward_backward with a timing record of every launch, for profiling.
+ * `events` holds 2*capacity cudaEvent_t created by the caller; launch i
+ * (i < capacity) is bracketed by events[2i] and events[2i+1], recorded on
+ * `stream`, and its flkl_launch_kind is written to the host array kinds[i].
+ * *n_launches (host) receives the number of launches of the call (which may
+ * exceed capacity; the extra ones are not recorded).  Same results and
+ * errors as flkl_forward_backward, plus FLKL_ERR_INVALID_ARG for a null
+ * events/kinds/n_launches or a negative capacity. */
+FLKL_API flkl_status flkl_forward_backward_profiled(
+    const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
+    int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
+    float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
+    void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
+    void** events, int* kinds, int capacity, int* n_launches);
+
 /* Synchronises `stream`, then returns the device status recorded by the last
  * flkl_forward_backward call that used `workspace` (FLKL_OK or
  * FLKL_ERR_TIMEOUT), or FLKL_ERR_CUDA if the copy or the synchronisation

@@ -17,6 +17,7 @@ import torch
 
 __all__ = [
     "FLKL_OK", "FlklError", "flkl_abi_version", "flkl_workspace_size", "flkl_forward_backward",
+    "flkl_forward_backward_profiled", "LAUNCH_KINDS",
     "flkl_device_status", "flkl_set_wait_limit_ms", "flkl_wait_selftest", "flkl_status_string",
     "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
 ]
@@ -63,6 +64,9 @@ def _lib():
             c.c_int, c.c_int, c.c_int,                           # dW db accum_fp32
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,      # loss dX dW db
             c.c_void_p, c.c_size_t, c.c_void_p]                  # ws bytes stream
+        lib.flkl_forward_backward_profiled.restype = c.c_int
+        lib.flkl_forward_backward_profiled.argtypes = list(lib.flkl_forward_backward.argtypes) + [
+            c.c_void_p, c.c_void_p, c.c_int, c.c_void_p]
         lib.flkl_device_status.restype = c.c_int
         lib.flkl_device_status.argtypes = [c.c_void_p, c.c_void_p]
         lib.flkl_set_wait_limit_ms.restype = None
@@ -99,6 +103,28 @@ def flkl_forward_backward(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtyp
         float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
         int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
         int(workspace_bytes), stream)
+
+
+LAUNCH_KINDS = ("prepare", "stats", "combine", "loss", "grad", "dW", "dX", "db", "zero")
+
+
+def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                                   temperature, eps, reduction, compute_dW, compute_db,
+                                   accum_fp32, loss, dX, dW, db, workspace, workspace_bytes,
+                                   stream, events, capacity):
+    """The profiled C entry point.  ``events`` is a list of 2*capacity
+    torch.cuda.Event(enable_timing=True); returns (status, kinds) where kinds
+    lists the launch kind of each recorded launch pair."""
+    c = ctypes
+    ev = (c.c_void_p * (2 * capacity))(*[e.cuda_event for e in events[:2 * capacity]])
+    kinds = (c.c_int * max(capacity, 1))()
+    n = c.c_int(0)
+    st = _lib().flkl_forward_backward_profiled(
+        X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
+        int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
+        int(workspace_bytes), stream, ev, kinds, int(capacity), c.byref(n))
+    return st, [kinds[i] for i in range(min(n.value, capacity))], n.value
 
 
 def flkl_device_status(workspace_ptr, stream=None) -> int:

@@ -165,6 +165,36 @@ TcGemmArgs gemm_args(long long M, long long N, long long K, int m_fastest, int* 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Optional per-launch event recording (flkl_forward_backward_profiled): an
+// event before and after every launch, on the launch stream, and the kind of
+// each launch.  A null recorder records nothing.
+struct Recorder {
+  cudaEvent_t* events;  // 2 * capacity events
+  int* kinds;           // capacity
+  int capacity;
+  int count;
+  cudaStream_t st;
+  void before(int kind) {
+    if (count < capacity) {
+      kinds[count] = kind;
+      cudaEventRecord(events[2 * count], st);
+    }
+  }
+  void after() {
+    if (count < capacity) cudaEventRecord(events[2 * count + 1], st);
+    ++count;
+  }
+};
+struct Rec {
+  Recorder* r;
+  Rec(Recorder* rr, int kind) : r(rr) {
+    if (r) r->before(kind);
+  }
+  ~Rec() {
+    if (r) r->after();
+  }
+};
+
 #define FLKL_CUDA(x)                               \
   do {                                             \
     if ((x) != cudaSuccess) return FLKL_ERR_CUDA;  \
@@ -174,7 +204,8 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
                    const __nv_bfloat16* b, const __nv_bfloat16* Q, const int64_t* labels,
                    long long ignore_index, int BT, int H, int V, float T, float eps,
                    int compute_dW, int compute_db, int accum_fp32, float* loss,
-                   __nv_bfloat16* dX, void* dW, void* db, uint8_t* ws, cudaStream_t st) {
+                   __nv_bfloat16* dX, void* dW, void* db, uint8_t* ws, cudaStream_t st,
+                   Recorder* rec) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
   float* rows = reinterpret_cast<float*>(ws + P.off_rows);
@@ -199,14 +230,21 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     TcGemmArgs g = gemm_args(BT, V, H, 1, err);
     EpiStats::Params ep{Q, b, BT, V, t_scale, eps, stats,
                         static_cast<long long>(P.n_tiles) * BT};
+    Rec r_(rec, 1);
     FLKL_CUDA((launch_tc<EpiStats, false, false>(mX_k, mW_k, g, ep, st)));
   }
-  k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
-      stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
-      coefQ, rowloss);
-  FLKL_CUDA(cudaGetLastError());
-  k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
-  FLKL_CUDA(cudaGetLastError());
+  {
+    Rec r_(rec, 2);
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
+        stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+        coefQ, rowloss);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  {
+    Rec r_(rec, 3);
+    k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
+    FLKL_CUDA(cudaGetLastError());
+  }
 
   const int ldg = static_cast<int>(P.Vc);
   for (long long c = 0; c < P.nchunks; ++c) {
@@ -217,6 +255,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
       TcGemmArgs g = gemm_args(BT, Vw, H, 1, err);
       g.b_n_off = c0;
       EpiGrad::Params ep{Q, b, BT, V, c0, ldg, G, t_scale, lse2, coefS, coefQ, dbpart};
+      Rec r_(rec, 4);
       FLKL_CUDA((launch_tc<EpiGrad, false, false>(mX_k, mW_k, g, ep, st)));
     }
     CUtensorMap mG_k, mG_mn;
@@ -225,6 +264,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     if (compute_dW) {
       TcGemmArgs g = gemm_args(Vw, H, BT, 0, err);
       EpiStoreRows::Params ep{dW, H, Vw, H, c0, accum_fp32};
+      Rec r_(rec, 5);
       FLKL_CUDA((launch_tc<EpiStoreRows, true, true>(mG_mn, mX_mn, g, ep, st)));
     }
     {
@@ -232,10 +272,12 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
       g.b_k_off = c0;
       int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
       EpiAccumRows::Params ep{dxpart, dX, H, BT, H, mode};
+      Rec r_(rec, 6);
       FLKL_CUDA((launch_tc<EpiAccumRows, false, true>(mG_k, mW_mn, g, ep, st)));
     }
   }
   if (compute_db) {
+    Rec r_(rec, 7);
     k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
         dbpart, static_cast<int>(P.db_groups), V, db, accum_fp32);
     FLKL_CUDA(cudaGetLastError());
@@ -246,7 +288,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
 flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* b, const float* Q,
                     const int64_t* labels, long long ignore_index, int BT, int H, int V, float T,
                     float eps, int compute_dW, int compute_db, float* loss, float* dX, float* dW,
-                    float* db, uint8_t* ws, cudaStream_t st) {
+                    float* db, uint8_t* ws, cudaStream_t st, Recorder* rec) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
   float* rows = reinterpret_cast<float*>(ws + P.off_rows);
@@ -260,25 +302,38 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
   const float t_scale = 1.4426950408889634f / T;
   const unsigned mt = static_cast<unsigned>(P.m_tiles);
 
+  {
+  Rec r_(rec, 1);
   k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
       X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT);
   FLKL_CUDA(cudaGetLastError());
-  k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
-      stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
-      coefQ, rowloss);
-  FLKL_CUDA(cudaGetLastError());
-  k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
-  FLKL_CUDA(cudaGetLastError());
+  }
+  {
+    Rec r_(rec, 2);
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
+        stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+        coefQ, rowloss);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  {
+    Rec r_(rec, 3);
+    k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
+    FLKL_CUDA(cudaGetLastError());
+  }
 
   const int ldg = static_cast<int>(P.Vc);
   for (long long c = 0; c < P.nchunks; ++c) {
     const int c0 = static_cast<int>(c * P.Vc);
     const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
+    {
+    Rec r_(rec, 4);
     k_simt_grad<<<dim3(static_cast<unsigned>(cdiv(Vw, ST_T)), mt), 256, 0, st>>>(
         X, W, b, Q, BT, H, V, c0, Vw, t_scale, lse2, coefS, coefQ, G, ldg, dbpart);
     FLKL_CUDA(cudaGetLastError());
+    }
     if (compute_dW) {
       // dW[c0 + v][h] = sum_r G[r][v] X[r][h]
+      Rec r_(rec, 5);
       k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)),
                              static_cast<unsigned>(cdiv(Vw, ST_T))),
                         256, 0, st>>>(G, 1, ldg, X, 1, H, Vw, H, BT, nullptr, dW, H, c0, 4);
@@ -286,11 +341,13 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
     }
     const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
     // dX[r][h] (+)= sum_v G[r][v] W[c0 + v][h]
+    Rec r_(rec, 6);
     k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)), mt), 256, 0, st>>>(
         G, ldg, 1, W + static_cast<size_t>(c0) * H, 1, H, BT, H, Vw, dxpart, dX, H, 0, mode);
     FLKL_CUDA(cudaGetLastError());
   }
   if (compute_db) {
+    Rec r_(rec, 7);
     k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
         dbpart, static_cast<int>(P.db_groups), V, db, 1);
     FLKL_CUDA(cudaGetLastError());
@@ -347,12 +404,17 @@ const char* flkl_status_string(int s) {
   }
 }
 
-flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, const void* Q,
+}  // extern "C"
+
+namespace flkl {
+namespace {
+
+flkl_status forward_backward_impl(const void* X, const void* W, const void* b, const void* Q,
                                   const int64_t* shift_labels, int64_t ignore_index, int64_t BT,
                                   int64_t H, int64_t V, int dtype, float temperature, float eps,
                                   int reduction, int compute_dW, int compute_db, int accum_fp32,
                                   float* loss, void* dX, void* dW, void* db, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
+                                  size_t workspace_bytes, void* stream, Recorder* rec) {
   // ---- scalar arguments
   if (dtype != FLKL_DTYPE_F32 && dtype != FLKL_DTYPE_BF16) return FLKL_ERR_INVALID_ARG;
   if (reduction == FLKL_REDUCTION_NONE) return FLKL_ERR_UNSUPPORTED;
@@ -385,12 +447,16 @@ flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, c
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int bt = static_cast<int>(BT), h = static_cast<int>(H), v = static_cast<int>(V);
 
-  k_prepare<<<1, 1024, 0, st>>>(shift_labels, bt, static_cast<long long>(ignore_index), reduction,
-                                v, temperature, reinterpret_cast<DevCtl*>(ws));
-  FLKL_CUDA(cudaGetLastError());
+  {
+    Rec r_(rec, 0);
+    k_prepare<<<1, 1024, 0, st>>>(shift_labels, bt, static_cast<long long>(ignore_index),
+                                  reduction, v, temperature, reinterpret_cast<DevCtl*>(ws));
+    FLKL_CUDA(cudaGetLastError());
+  }
 
   if (BT == 0) {
     // No rows: loss 0, and zero parameter gradients when asked for.
+    Rec r_(rec, 8);
     k_zero<<<1, 32, 0, st>>>(loss, sizeof(float));
     FLKL_CUDA(cudaGetLastError());
     const size_t pe = (dtype == FLKL_DTYPE_F32 || accum_fp32) ? 4 : 2;
@@ -411,13 +477,46 @@ flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, c
     return run_tc(P, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
                   static_cast<const __nv_bfloat16*>(b), static_cast<const __nv_bfloat16*>(Q),
                   shift_labels, ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db,
-                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st);
+                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st, rec);
   }
   return run_f32(P, static_cast<const float*>(X), static_cast<const float*>(W),
                  static_cast<const float*>(b), static_cast<const float*>(Q), shift_labels,
                  ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db, loss,
                  static_cast<float*>(dX), static_cast<float*>(dW), static_cast<float*>(db), ws,
-                 st);
+                 st, rec);
+}
+
+}  // namespace
+}  // namespace flkl
+
+extern "C" {
+
+flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, const void* Q,
+                                  const int64_t* shift_labels, int64_t ignore_index, int64_t BT,
+                                  int64_t H, int64_t V, int dtype, float temperature, float eps,
+                                  int reduction, int compute_dW, int compute_db, int accum_fp32,
+                                  float* loss, void* dX, void* dW, void* db, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                               temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr);
+}
+
+flkl_status flkl_forward_backward_profiled(
+    const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
+    int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
+    float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
+    void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
+    void** events, int* kinds, int capacity, int* n_launches) {
+  if (events == nullptr || kinds == nullptr || n_launches == nullptr || capacity < 0)
+    return FLKL_ERR_INVALID_ARG;
+  Recorder r{reinterpret_cast<cudaEvent_t*>(events), kinds, capacity, 0,
+             static_cast<cudaStream_t>(stream)};
+  const flkl_status s = forward_backward_impl(
+      X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype, temperature, eps, reduction,
+      compute_dW, compute_db, accum_fp32, loss, dX, dW, db, workspace, workspace_bytes, stream, &r);
+  *n_launches = r.count;
+  return s;
 }
 
 flkl_status flkl_device_status(const void* workspace, void* stream) {

@@ -220,3 +220,36 @@ def test_no_bt_by_v_allocation_at_full_size():
     torch.cuda.synchronize()
     assert torch.cuda.max_memory_allocated(dev) - base == 0
     assert r["workspace"].numel() < w.BT * w.V * 2 // 4
+
+
+def test_profiled_entry_records_every_launch_and_matches():
+    """flkl_forward_backward_profiled gives the same results as the plain
+    entry and tags every launch with its kind, in launch order."""
+    w = small_case(dtype="bf16", BT=130, H=128, V=2056, bias=True)
+    inp = make_inputs(w)
+    dev = torch.device("cuda:0")
+    ref = run_gpu(inp)
+    g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    out = {k: torch.empty_like(ref[k]) for k in ("loss", "dX", "dW", "db")}
+    ws = torch.empty_like(ref["workspace"])
+    stream = torch.cuda.current_stream()
+    cap = 64
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
+    for e in events:
+        e.record(stream)
+    p = lambda t: None if t is None else t.data_ptr()
+    st, kinds, n = pkg.flkl_forward_backward_profiled(
+        p(g["X"]), p(g["W"]), p(g["b"]), p(g["Q"]), None, -100, w.BT, w.H, w.V, 1, 1.0, 1e-10, 0,
+        1, 1, 1, p(out["loss"]), p(out["dX"]), p(out["dW"]), p(out["db"]), p(ws), ws.numel(),
+        stream.cuda_stream, events, cap)
+    torch.cuda.synchronize()
+    assert st == 0 and n == len(kinds)
+    names = [pkg.LAUNCH_KINDS[k] for k in kinds]
+    nchunks = names.count("grad")
+    assert nchunks >= 2
+    assert names == (["prepare", "stats", "combine", "loss"] + ["grad", "dW", "dX"] * nchunks
+                     + ["db"])
+    for i in range(n):
+        assert events[2 * i].elapsed_time(events[2 * i + 1]) >= 0.0
+    for k in ("loss", "dX", "dW", "db"):
+        assert torch.equal(out[k], ref[k]), k
