@@ -73,7 +73,8 @@ typedef enum {
   FLKL_ERR_UNSUPPORTED = 2, /* reduction NONE, misalignment, size limits     */
   FLKL_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed          */
   FLKL_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out (kernel quit)  */
-  FLKL_ERR_WORKSPACE = 5    /* workspace missing, misaligned or too small    */
+  FLKL_ERR_WORKSPACE = 5,   /* workspace missing, misaligned or too small    */
+  FLKL_ERR_TOO_LARGE = 6    /* sizes need more than FLKL_NOALLOC_SCRATCH_BYTES */
 } flkl_status;
 
 /* Version of this ABI (FLKL_ABI_VERSION of the built library). */
@@ -150,6 +151,42 @@ FLKL_API flkl_status flkl_forward_backward_profiled(
     float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
     void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
     void** events, int* kinds, int capacity, int* n_launches);
+
+/* Size of the fixed device scratch used by flkl_forward_backward_noalloc. */
+#define FLKL_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* flkl_forward_backward for callers that cannot allocate device memory.
+ *
+ * No counterpart on the pages: this is a library convenience.  Some callers
+ * cannot call cudaMalloc or hand over a workspace: code that runs inside a
+ * host framework whose allocator owns every device byte (a plugin or
+ * extension interface that passes in tensors but no scratch), or a
+ * latency-critical loop where cudaMalloc's implicit device synchronisation
+ * is not acceptable.  This entry point takes the same arguments minus the
+ * workspace and uses a fixed scratch array of FLKL_NOALLOC_SCRATCH_BYTES
+ * (64 MiB) that lives in the library itself: every GPU that loads the
+ * library holds those 64 MiB until the process exits.  The caller still
+ * passes every input and output.
+ *
+ *  - It allocates nothing and calls no allocating routine.
+ *  - Sizes whose flkl_workspace_size() exceeds FLKL_NOALLOC_SCRATCH_BYTES
+ *    return FLKL_ERR_TOO_LARGE before any launch (BT=1024, H=4096,
+ *    V=128256 with dW needs 57.3 MiB and fits).
+ *  - The first call on a device looks up the scratch address on that device
+ *    (the device must be current); make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the one scratch array, which keeps the
+ *    previous call's contents (the call initialises what it reads).  Calls
+ *    that can overlap on the GPU (different streams, or different host
+ *    threads) race on it and give wrong results: serialise them.
+ *  - A device-side wait that runs out is recorded in the shared scratch and
+ *    cannot be read back through this entry point; use
+ *    flkl_forward_backward with a workspace when that status is needed. */
+FLKL_API flkl_status flkl_forward_backward_noalloc(
+    const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
+    int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
+    float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
+    void* dX, void* dW, void* db, void* stream);
 
 /* Synchronises `stream`, then returns the device status recorded by the last
  * flkl_forward_backward call that used `workspace` (FLKL_OK or

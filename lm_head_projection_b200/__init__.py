@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "FLKL_OK", "FlklError", "flkl_abi_version", "flkl_workspace_size", "flkl_forward_backward",
-    "flkl_forward_backward_profiled", "LAUNCH_KINDS",
+    "flkl_forward_backward_profiled", "LAUNCH_KINDS", "flkl_forward_backward_noalloc",
     "flkl_device_status", "flkl_set_wait_limit_ms", "flkl_wait_selftest", "flkl_status_string",
     "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
 ]
@@ -67,6 +67,9 @@ def _lib():
         lib.flkl_forward_backward_profiled.restype = c.c_int
         lib.flkl_forward_backward_profiled.argtypes = list(lib.flkl_forward_backward.argtypes) + [
             c.c_void_p, c.c_void_p, c.c_int, c.c_void_p]
+        lib.flkl_forward_backward_noalloc.restype = c.c_int
+        lib.flkl_forward_backward_noalloc.argtypes = (
+            list(lib.flkl_forward_backward.argtypes[:20]) + [c.c_void_p])
         lib.flkl_device_status.restype = c.c_int
         lib.flkl_device_status.argtypes = [c.c_void_p, c.c_void_p]
         lib.flkl_set_wait_limit_ms.restype = None
@@ -103,6 +106,18 @@ def flkl_forward_backward(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtyp
         float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
         int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
         int(workspace_bytes), stream)
+
+
+def flkl_forward_backward_noalloc(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                                  temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
+                                  loss, dX, dW, db, stream) -> int:
+    """The allocation-free C entry point (raw pointers, no workspace): it
+    uses the library's fixed 64 MiB device scratch, for callers that cannot
+    allocate device memory.  Returns the status (6 = sizes too large)."""
+    return _lib().flkl_forward_backward_noalloc(
+        X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
+        int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, stream)
 
 
 LAUNCH_KINDS = ("prepare", "stats", "combine", "loss", "grad", "dW", "dX", "db", "zero")

@@ -400,6 +400,7 @@ const char* flkl_status_string(int s) {
     case FLKL_ERR_CUDA: return "CUDA runtime error";
     case FLKL_ERR_TIMEOUT: return "a device-side wait ran out of time";
     case FLKL_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case FLKL_ERR_TOO_LARGE: return "sizes need more scratch than the fixed 64 MiB device scratch";
     default: return "unknown status";
   }
 }
@@ -486,10 +487,59 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
                  st, rec);
 }
 
+// Fixed scratch of flkl_forward_backward_noalloc (see flkl.h): part of the
+// library's device image, so it exists on every device that loads the
+// library, without any allocation call.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FLKL_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the fixed scratch on the current device, looked up once
+// per device.  In host code the symbol is only a host-side handle: the
+// address a kernel may use comes from cudaGetSymbolAddress.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 }  // namespace flkl
 
 extern "C" {
+
+flkl_status flkl_forward_backward_noalloc(const void* X, const void* W, const void* b,
+                                          const void* Q, const int64_t* shift_labels,
+                                          int64_t ignore_index, int64_t BT, int64_t H, int64_t V,
+                                          int dtype, float temperature, float eps, int reduction,
+                                          int compute_dW, int compute_db, int accum_fp32,
+                                          float* loss, void* dX, void* dW, void* db,
+                                          void* stream) {
+  const size_t need = flkl_workspace_size(BT, H, V, dtype, compute_dW, compute_db);
+  if (need == 0) {
+    // invalid sizes or dtype: let the regular validation name the error
+    return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                                 temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
+                                 loss, dX, dW, db, nullptr, 0, stream, nullptr);
+  }
+  if (need > FLKL_NOALLOC_SCRATCH_BYTES) return FLKL_ERR_TOO_LARGE;
+  void* scratch = nullptr;
+  if (noalloc_scratch(&scratch) != cudaSuccess) return FLKL_ERR_CUDA;
+  return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                               temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, scratch, FLKL_NOALLOC_SCRATCH_BYTES, stream,
+                               nullptr);
+}
 
 flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, const void* Q,
                                   const int64_t* shift_labels, int64_t ignore_index, int64_t BT,
