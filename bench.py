@@ -43,7 +43,6 @@ from lm_head_projection_b200.workloads import HEADLINE, WORKLOADS, make_inputs  
 
 METRIC = "fwd+bwd tokens/s at H=4096,V=128256 bf16; % of roofline (tensor/HBM)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GEMM_KINDS = {"stats", "grad", "dW", "dX"}
 
 
 def load_peaks():
@@ -242,46 +241,42 @@ def run_ours(args):
     for e in events:  # torch creates the CUDA event on its first record
         e.record(stream)
     torch.cuda.synchronize()
-    per_kind = {}
+    per_kind = {}  # kind -> [ms, launches, gemm flops]
     launches_per_step = 0
-    kernel_flops = {}
     for _ in range(args.steps):
-        st, kinds, n = pkg.flkl_forward_backward_profiled(*call_args, events, cap)
+        st, kinds, flops, n = pkg.flkl_forward_backward_profiled(*call_args, events, cap)
         if st != 0:
             raise pkg.FlklError(st, "flkl_forward_backward_profiled")
         launches_per_step = n
         torch.cuda.synchronize()
         for i, k in enumerate(kinds):
-            name = pkg.LAUNCH_KINDS[k]
-            d = per_kind.setdefault(name, [0.0, 0])
+            d = per_kind.setdefault(pkg.LAUNCH_KINDS[k], [0.0, 0, 0.0])
             d[0] += events[2 * i].elapsed_time(events[2 * i + 1])
             d[1] += 1
+            d[2] += flops[i]
     clocks.stop()
     clk = clocks.summary()
 
-    # GEMM FLOPs per step of each kind (2*M*N*K summed over its launches)
-    base = 2.0 * w.BT * w.H * w.V
-    kernel_flops = {"stats": base, "grad": base, "dX": base,
-                    "dW": base if inp["compute_dW"] else 0.0}
     total_prof_ms = sum(v[0] for v in per_kind.values())
     dominant = max(per_kind, key=lambda k: per_kind[k][0])
     peaks, peaks_src = load_peaks()
     peak_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    dom_ms, dom_n = per_kind[dominant]
-    if dominant in GEMM_KINDS:
-        launches_of_kind_per_step = dom_n / args.steps
-        flops_per_launch = kernel_flops[dominant] / launches_of_kind_per_step
-        achieved = flops_per_launch / (dom_ms / dom_n * 1e-3) / 1e12
+    dom_ms, dom_n, dom_flops = per_kind[dominant]
+    if dom_flops > 0:
+        achieved = dom_flops / (dom_ms * 1e-3) / 1e12  # = flops per launch / avg launch time
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_sust,
                     "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4), "traffic": None,
-                    "kernel": f"tc_gemm_kernel<{dominant}>",
+                    "kernel": f"tc_group_kernel ({dominant} launches)",
+                    "flops_per_launch": dom_flops / dom_n,
+                    "avg_launch_ms": round(dom_ms / dom_n, 4),
                     "peak_note": f"bf16_tflops_sustained of {peaks_src}",
                     "share": round(dom_ms / total_prof_ms, 3)}
     else:
         roofline = {"bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": None, "traffic": None, "kernel": dominant}
     breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step":
-                     round(v[1] / args.steps, 2), "share": round(v[0] / total_prof_ms, 3)}
+                     round(v[1] / args.steps, 2), "share": round(v[0] / total_prof_ms, 3),
+                     "tflops": round(v[2] / (v[0] * 1e-3) / 1e12, 1) if v[2] else None}
                  for k, v in sorted(per_kind.items())}
 
     ms_per_step = ms / args.steps

@@ -130,30 +130,34 @@ typedef enum {
   FLKL_LAUNCH_STATS = 1,    /* pass 1: logits GEMM + softmax/KL statistics    */
   FLKL_LAUNCH_COMBINE = 2,  /* per-row log-sum-exp and row loss              */
   FLKL_LAUNCH_LOSS = 3,     /* reduction of the row losses                   */
-  FLKL_LAUNCH_GRAD = 4,     /* pass 2: logits GEMM again + G to staging      */
-  FLKL_LAUNCH_DW = 5,       /* dW chunk GEMM                                 */
-  FLKL_LAUNCH_DX = 6,       /* dX chunk GEMM                                 */
+  FLKL_LAUNCH_GRAD = 4,     /* pass 2 of one chunk: logits again + G staging */
+  FLKL_LAUNCH_DW = 5,       /* dW chunk GEMM (fp32 path)                     */
+  FLKL_LAUNCH_DX = 6,       /* dX chunk GEMM (fp32 path)                     */
   FLKL_LAUNCH_DB = 7,       /* db column reduction                           */
-  FLKL_LAUNCH_ZERO = 8      /* zero fill (BT = 0)                            */
+  FLKL_LAUNCH_ZERO = 8,     /* zero fill (BT = 0)                            */
+  FLKL_LAUNCH_CHUNK = 9     /* bf16 path, one per vocabulary chunk c: dX(c), */
+                            /* pass 2 of chunk c+1 and dW(c) in one launch   */
 } flkl_launch_kind;
 
 /* flkl_forward_backward with a timing record of every launch, for profiling.
  * `events` holds 2*capacity cudaEvent_t created by the caller; launch i
  * (i < capacity) is bracketed by events[2i] and events[2i+1], recorded on
- * `stream`, and its flkl_launch_kind is written to the host array kinds[i].
- * *n_launches (host) receives the number of launches of the call (which may
- * exceed capacity; the extra ones are not recorded).  Same results and
- * errors as flkl_forward_backward, plus FLKL_ERR_INVALID_ARG for a null
- * events/kinds/n_launches or a negative capacity. */
+ * `stream`; its flkl_launch_kind is written to the host array kinds[i] and
+ * its GEMM FLOPs (2*M*N*K summed over the launch's problems, 0 for launches
+ * without a GEMM) to the host array flops[i].  *n_launches (host) receives
+ * the number of launches of the call (which may exceed capacity; the extra
+ * ones are not recorded).  Same results and errors as
+ * flkl_forward_backward, plus FLKL_ERR_INVALID_ARG for a null
+ * events/kinds/flops/n_launches or a negative capacity. */
 FLKL_API flkl_status flkl_forward_backward_profiled(
     const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
     int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
     float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
     void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
-    void** events, int* kinds, int capacity, int* n_launches);
+    void** events, int* kinds, double* flops, int capacity, int* n_launches);
 
 /* Size of the fixed device scratch used by flkl_forward_backward_noalloc. */
-#define FLKL_NOALLOC_SCRATCH_BYTES (64u << 20)
+#define FLKL_NOALLOC_SCRATCH_BYTES (128u << 20)
 
 /* flkl_forward_backward for callers that cannot allocate device memory.
  *
@@ -164,14 +168,14 @@ FLKL_API flkl_status flkl_forward_backward_profiled(
  * latency-critical loop where cudaMalloc's implicit device synchronisation
  * is not acceptable.  This entry point takes the same arguments minus the
  * workspace and uses a fixed scratch array of FLKL_NOALLOC_SCRATCH_BYTES
- * (64 MiB) that lives in the library itself: every GPU that loads the
- * library holds those 64 MiB until the process exits.  The caller still
+ * (128 MiB) that lives in the library itself: every GPU that loads the
+ * library holds those 128 MiB until the process exits.  The caller still
  * passes every input and output.
  *
  *  - It allocates nothing and calls no allocating routine.
  *  - Sizes whose flkl_workspace_size() exceeds FLKL_NOALLOC_SCRATCH_BYTES
  *    return FLKL_ERR_TOO_LARGE before any launch (BT=1024, H=4096,
- *    V=128256 with dW needs 57.3 MiB and fits).
+ *    V=128256 with dW needs 98.6 MiB and fits).
  *  - The first call on a device looks up the scratch address on that device
  *    (the device must be current); make that first call before any stream
  *    capture.

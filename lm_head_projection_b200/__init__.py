@@ -66,7 +66,7 @@ def _lib():
             c.c_void_p, c.c_size_t, c.c_void_p]                  # ws bytes stream
         lib.flkl_forward_backward_profiled.restype = c.c_int
         lib.flkl_forward_backward_profiled.argtypes = list(lib.flkl_forward_backward.argtypes) + [
-            c.c_void_p, c.c_void_p, c.c_int, c.c_void_p]
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_void_p]
         lib.flkl_forward_backward_noalloc.restype = c.c_int
         lib.flkl_forward_backward_noalloc.argtypes = (
             list(lib.flkl_forward_backward.argtypes[:20]) + [c.c_void_p])
@@ -112,7 +112,7 @@ def flkl_forward_backward_noalloc(X, W, b, Q, shift_labels, ignore_index, BT, H,
                                   temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
                                   loss, dX, dW, db, stream) -> int:
     """The allocation-free C entry point (raw pointers, no workspace): it
-    uses the library's fixed 64 MiB device scratch, for callers that cannot
+    uses the library's fixed 128 MiB device scratch, for callers that cannot
     allocate device memory.  Returns the status (6 = sizes too large)."""
     return _lib().flkl_forward_backward_noalloc(
         X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
@@ -120,7 +120,8 @@ def flkl_forward_backward_noalloc(X, W, b, Q, shift_labels, ignore_index, BT, H,
         int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, stream)
 
 
-LAUNCH_KINDS = ("prepare", "stats", "combine", "loss", "grad", "dW", "dX", "db", "zero")
+LAUNCH_KINDS = ("prepare", "stats", "combine", "loss", "grad", "dW", "dX", "db", "zero",
+                "chunk")
 
 
 def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
@@ -128,18 +129,21 @@ def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H
                                    accum_fp32, loss, dX, dW, db, workspace, workspace_bytes,
                                    stream, events, capacity):
     """The profiled C entry point.  ``events`` is a list of 2*capacity
-    torch.cuda.Event(enable_timing=True); returns (status, kinds) where kinds
-    lists the launch kind of each recorded launch pair."""
+    torch.cuda.Event(enable_timing=True), each recorded once beforehand (torch
+    creates the CUDA event lazily).  Returns (status, kinds, flops, n) with the
+    launch kind and GEMM FLOPs of each recorded launch and the launch count."""
     c = ctypes
     ev = (c.c_void_p * (2 * capacity))(*[e.cuda_event for e in events[:2 * capacity]])
     kinds = (c.c_int * max(capacity, 1))()
+    flops = (c.c_double * max(capacity, 1))()
     n = c.c_int(0)
     st = _lib().flkl_forward_backward_profiled(
         X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
         float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
         int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
-        int(workspace_bytes), stream, ev, kinds, int(capacity), c.byref(n))
-    return st, [kinds[i] for i in range(min(n.value, capacity))], n.value
+        int(workspace_bytes), stream, ev, kinds, flops, int(capacity), c.byref(n))
+    k = min(n.value, capacity)
+    return st, [kinds[i] for i in range(k)], [flops[i] for i in range(k)], n.value
 
 
 def flkl_device_status(workspace_ptr, stream=None) -> int:

@@ -40,9 +40,12 @@ struct Plan {
   bool tc;
   int tile_m, tile_n;
   long long m_tiles, n_tiles;  // pass tiles over [BT] x [V]
+  long long n_stat;            // column groups of the pass-1 statistics
   long long Vc, nchunks;
   long long db_groups;
-  size_t off_st, off_rows, off_G, off_dx, off_db, total;
+  long long n_counters;  // tile counters of the persistent launches
+  size_t off_cnt, off_st, off_rows, off_G, off_dx, off_db, total;
+  size_t g_stride;       // bytes between the two G staging buffers
 };
 
 bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int compute_db,
@@ -57,6 +60,7 @@ bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int 
   const size_t elem = p.tc ? 2 : 4;
   p.m_tiles = cdiv(BT, p.tile_m);
   p.n_tiles = cdiv(V, p.tile_n);
+  p.n_stat = p.tc ? cdiv(V, TC_EPI_COLS) : p.n_tiles;
   // Chunk width: at most V/8 (rounded up to the tile width) and at most the
   // staging budget; never below one tile.
   long long vc = cdiv(cdiv(V, 8), p.tile_n) * p.tile_n;
@@ -68,14 +72,20 @@ bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int 
   vc = std::min(vc, p.n_tiles * p.tile_n);
   p.Vc = vc;
   p.nchunks = cdiv(V, vc);
-  p.db_groups = p.tc ? p.m_tiles * 4 : p.m_tiles;
+  p.db_groups = p.tc ? p.m_tiles * (TC_BM / 32) : p.m_tiles;
   size_t off = align256(sizeof(DevCtl));
+  p.n_counters = p.nchunks + 2;
+  p.off_cnt = off;
+  off += align256(size_t(p.n_counters) * 4);
   p.off_st = off;
-  off += align256(size_t(5) * p.n_tiles * BT * 4);
+  off += align256(size_t(5) * p.n_stat * BT * 4);
   p.off_rows = off;
   off += align256(size_t(4) * BT * 4);
   p.off_G = off;
-  off += align256(size_t(BT) * vc * elem);
+  // two staging buffers on the tensor-core path: chunk c+1's gradient block
+  // is produced while chunk c's is consumed
+  p.g_stride = align256(size_t(BT) * vc * elem);
+  off += p.g_stride * ((p.tc && p.nchunks > 1) ? 2 : 1);
   p.off_dx = off;
   if (p.nchunks > 1) off += align256(size_t(BT) * H * 4);
   p.off_db = off;
@@ -129,38 +139,45 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
-template <class Epi, bool A_MN, bool B_MN>
-cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmArgs& g,
-                      const typename Epi::Params& ep, cudaStream_t st) {
-  auto kern = tc_gemm_kernel<Epi, A_MN, B_MN>;
+cudaError_t launch_group(const TcMaps& maps, const TcLaunch& L, cudaStream_t st) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(tc_group_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const long long tiles = static_cast<long long>(g.m_tiles) * g.n_tiles;
-  if (tiles <= 0) return cudaSuccess;
-  const int grid = static_cast<int>(std::min<long long>(tiles, num_sms()));
-  kern<<<grid, TC_THREADS, TC_SMEM_BYTES, st>>>(ta, tb, g, ep);
+  if (L.total_tiles <= 0) return cudaSuccess;
+  // one CTA pair (cluster of 2) per claimed tile, at most one CTA per SM
+  const int grid = 2 * static_cast<int>(std::min<long long>(L.total_tiles, num_sms() / 2));
+  tc_group_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, st>>>(maps, L);
   return cudaGetLastError();
 }
 
-TcGemmArgs gemm_args(long long M, long long N, long long K, int m_fastest, int* err) {
-  TcGemmArgs g{};
-  g.M = static_cast<int>(M);
-  g.N = static_cast<int>(N);
-  g.K = static_cast<int>(K);
-  g.m_tiles = static_cast<int>(cdiv(M, TC_BM));
-  g.n_tiles = static_cast<int>(cdiv(N, TC_BN));
-  g.num_kb = static_cast<int>(cdiv(K, TC_BK));
-  g.m_fastest = m_fastest;
-  g.err_flag = err;
-  g.wait_limit_ns = g_wait_limit_ns;
-  return g;
+// Appends a problem D[M,N] (K deep) of `kind` to launch L; A and B are its
+// tensor maps.  Returns false when L is full.
+bool add_problem(TcLaunch& L, TcMaps& maps, int kind, long long M, long long N, long long K,
+                 int m_fastest, const CUtensorMap& A, const CUtensorMap& B, int a_k_off = 0,
+                 int b_n_off = 0, int b_k_off = 0) {
+  if (L.nprob >= TC_MAX_PROBLEMS) return false;
+  TcProblem& P = L.prob[L.nprob];
+  P = TcProblem{};
+  P.kind = kind;
+  P.m_tiles = static_cast<int>(cdiv(M, TC_BM));
+  P.n_tiles = static_cast<int>(cdiv(N, TC_BN));
+  P.num_kb = static_cast<int>(cdiv(K, TC_BK));
+  P.m_fastest = m_fastest;
+  P.a_k_off = a_k_off;
+  P.b_n_off = b_n_off;
+  P.b_k_off = b_k_off;
+  P.tile_begin = L.total_tiles;
+  maps.m[2 * L.nprob] = A;
+  maps.m[2 * L.nprob + 1] = B;
+  L.total_tiles += P.m_tiles * P.n_tiles;
+  ++L.nprob;
+  return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -171,12 +188,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct Recorder {
   cudaEvent_t* events;  // 2 * capacity events
   int* kinds;           // capacity
+  double* flops;        // capacity: GEMM FLOPs of each launch (0 for the others)
   int capacity;
   int count;
   cudaStream_t st;
-  void before(int kind) {
+  void before(int kind, double f) {
     if (count < capacity) {
       kinds[count] = kind;
+      flops[count] = f;
       cudaEventRecord(events[2 * count], st);
     }
   }
@@ -187,8 +206,8 @@ struct Recorder {
 };
 struct Rec {
   Recorder* r;
-  Rec(Recorder* rr, int kind) : r(rr) {
-    if (r) r->before(kind);
+  Rec(Recorder* rr, int kind, double flops = 0.0) : r(rr) {
+    if (r) r->before(kind, flops);
   }
   ~Rec() {
     if (r) r->after();
@@ -207,36 +226,59 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
                    __nv_bfloat16* dX, void* dW, void* db, uint8_t* ws, cudaStream_t st,
                    Recorder* rec) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
+  int* counters = reinterpret_cast<int*>(ws + P.off_cnt);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
   float* rows = reinterpret_cast<float*>(ws + P.off_rows);
   float* lse2 = rows;
   float* coefS = rows + BT;
   float* coefQ = rows + 2 * static_cast<size_t>(BT);
   float* rowloss = rows + 3 * static_cast<size_t>(BT);
-  __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(ws + P.off_G);
+  __nv_bfloat16* Gbuf[2] = {reinterpret_cast<__nv_bfloat16*>(ws + P.off_G),
+                            reinterpret_cast<__nv_bfloat16*>(ws + P.off_G + P.g_stride)};
   float* dxpart = reinterpret_cast<float*>(ws + P.off_dx);
   float* dbpart = compute_db ? reinterpret_cast<float*>(ws + P.off_db) : nullptr;
-  int* err = &ctl->err;
   const float LOG2E = 1.4426950408889634f;
   const float t_scale = LOG2E / T;
+  const int ldg = static_cast<int>(P.Vc);
 
   CUtensorMap mX_k, mW_k, mX_mn, mW_mn;
-  if (!make_map(&mX_k, X, H, BT, H, TC_BM) || !make_map(&mW_k, W, H, V, H, TC_BN) ||
-      !make_map(&mX_mn, X, H, BT, H, 64) || !make_map(&mW_mn, W, H, V, H, 64))
+  if (!make_map(&mX_k, X, H, BT, H, TC_HM) || !make_map(&mW_k, W, H, V, H, TC_HM) ||
+      !make_map(&mX_mn, X, H, BT, H, TC_BK) || !make_map(&mW_mn, W, H, V, H, TC_BK))
     return FLKL_ERR_CUDA;
+
+  auto new_launch = [&](int counter_index) {
+    TcLaunch L{};
+    L.counter = counters + counter_index;
+    L.err_flag = &ctl->err;
+    L.wait_limit_ns = g_wait_limit_ns;
+    L.stats = EpiStats::Params{Q, b, BT, V, t_scale, eps, stats,
+                               static_cast<long long>(P.n_stat) * BT};
+    return L;
+  };
+  auto chunk_c0 = [&](long long c) { return static_cast<int>(c * P.Vc); };
+  auto chunk_w = [&](long long c) {
+    return static_cast<int>(std::min<long long>(P.Vc, V - c * P.Vc));
+  };
+  // pass-2 problem of chunk c: logits of the chunk again -> G staging
+  auto add_grad = [&](TcLaunch& L, TcMaps& maps, long long c) {
+    const int c0 = chunk_c0(c);
+    L.grad = EpiGrad::Params{Q,     b,     BT,   V,     c0,     ldg,   Gbuf[c & 1],
+                             t_scale, lse2, coefS, coefQ, dbpart};
+    return add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, c0, 0);
+  };
 
   // pass 1: statistics over all V
   {
-    TcGemmArgs g = gemm_args(BT, V, H, 1, err);
-    EpiStats::Params ep{Q, b, BT, V, t_scale, eps, stats,
-                        static_cast<long long>(P.n_tiles) * BT};
-    Rec r_(rec, 1);
-    FLKL_CUDA((launch_tc<EpiStats, false, false>(mX_k, mW_k, g, ep, st)));
+    TcLaunch L = new_launch(0);
+    TcMaps maps{};
+    add_problem(L, maps, KIND_STATS, BT, V, H, 1, mX_k, mW_k);
+    Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
+    FLKL_CUDA(launch_group(maps, L, st));
   }
   {
     Rec r_(rec, 2);
-    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
-        stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
+        stats, static_cast<int>(P.n_stat), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
         coefQ, rowloss);
     FLKL_CUDA(cudaGetLastError());
   }
@@ -245,36 +287,37 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
     FLKL_CUDA(cudaGetLastError());
   }
-
-  const int ldg = static_cast<int>(P.Vc);
+  // pass 2 of chunk 0 alone
+  {
+    TcLaunch L = new_launch(1);
+    TcMaps maps{};
+    add_grad(L, maps, 0);
+    Rec r_(rec, 4, 2.0 * BT * static_cast<double>(chunk_w(0)) * H);
+    FLKL_CUDA(launch_group(maps, L, st));
+  }
+  // then one launch per chunk c: dX(c) (longest tiles first), pass 2 of
+  // chunk c+1 into the other staging buffer, dW(c) (shortest tiles last)
   for (long long c = 0; c < P.nchunks; ++c) {
-    const int c0 = static_cast<int>(c * P.Vc);
-    const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
-    // pass 2: gradient of the chunk's logits -> bf16 staging
-    {
-      TcGemmArgs g = gemm_args(BT, Vw, H, 1, err);
-      g.b_n_off = c0;
-      EpiGrad::Params ep{Q, b, BT, V, c0, ldg, G, t_scale, lse2, coefS, coefQ, dbpart};
-      Rec r_(rec, 4);
-      FLKL_CUDA((launch_tc<EpiGrad, false, false>(mX_k, mW_k, g, ep, st)));
-    }
+    const int c0 = chunk_c0(c), Vw = chunk_w(c);
+    __nv_bfloat16* G = Gbuf[c & 1];
     CUtensorMap mG_k, mG_mn;
-    if (!make_map(&mG_k, G, Vw, BT, ldg, TC_BM) || !make_map(&mG_mn, G, Vw, BT, ldg, 64))
+    if (!make_map(&mG_k, G, Vw, BT, ldg, TC_HM) || !make_map(&mG_mn, G, Vw, BT, ldg, TC_BK))
       return FLKL_ERR_CUDA;
+    TcLaunch L = new_launch(static_cast<int>(2 + c));
+    TcMaps maps{};
+    const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
+    L.dx = EpiAccumRows::Params{dxpart, dX, H, BT, H, mode};
+    add_problem(L, maps, KIND_DX, BT, H, Vw, 0, mG_k, mW_mn, 0, 0, c0);
+    if (c + 1 < P.nchunks) add_grad(L, maps, c + 1);
     if (compute_dW) {
-      TcGemmArgs g = gemm_args(Vw, H, BT, 0, err);
-      EpiStoreRows::Params ep{dW, H, Vw, H, c0, accum_fp32};
-      Rec r_(rec, 5);
-      FLKL_CUDA((launch_tc<EpiStoreRows, true, true>(mG_mn, mX_mn, g, ep, st)));
+      L.dw = EpiStoreRows::Params{dW, H, Vw, H, c0, accum_fp32};
+      add_problem(L, maps, KIND_DW, Vw, H, BT, 0, mG_mn, mX_mn);
     }
-    {
-      TcGemmArgs g = gemm_args(BT, H, Vw, 0, err);
-      g.b_k_off = c0;
-      int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
-      EpiAccumRows::Params ep{dxpart, dX, H, BT, H, mode};
-      Rec r_(rec, 6);
-      FLKL_CUDA((launch_tc<EpiAccumRows, false, true>(mG_k, mW_mn, g, ep, st)));
-    }
+    L.mix = 0;  // problems in sequence (interleaving pass-2 and dW tiles measured slower)
+    double f = 2.0 * BT * static_cast<double>(Vw) * H * (1 + (compute_dW ? 1 : 0));
+    if (c + 1 < P.nchunks) f += 2.0 * BT * static_cast<double>(chunk_w(c + 1)) * H;
+    Rec r_(rec, 9, f);
+    FLKL_CUDA(launch_group(maps, L, st));
   }
   if (compute_db) {
     Rec r_(rec, 7);
@@ -303,15 +346,15 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
   const unsigned mt = static_cast<unsigned>(P.m_tiles);
 
   {
-  Rec r_(rec, 1);
+  Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
   k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
       X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT);
   FLKL_CUDA(cudaGetLastError());
   }
   {
     Rec r_(rec, 2);
-    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 256, 0, st>>>(
-        stats, static_cast<int>(P.n_tiles), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
+        stats, static_cast<int>(P.n_stat), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
         coefQ, rowloss);
     FLKL_CUDA(cudaGetLastError());
   }
@@ -326,14 +369,14 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
     const int c0 = static_cast<int>(c * P.Vc);
     const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
     {
-    Rec r_(rec, 4);
+    Rec r_(rec, 4, 2.0 * BT * static_cast<double>(Vw) * H);
     k_simt_grad<<<dim3(static_cast<unsigned>(cdiv(Vw, ST_T)), mt), 256, 0, st>>>(
         X, W, b, Q, BT, H, V, c0, Vw, t_scale, lse2, coefS, coefQ, G, ldg, dbpart);
     FLKL_CUDA(cudaGetLastError());
     }
     if (compute_dW) {
       // dW[c0 + v][h] = sum_r G[r][v] X[r][h]
-      Rec r_(rec, 5);
+      Rec r_(rec, 5, 2.0 * BT * static_cast<double>(Vw) * H);
       k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)),
                              static_cast<unsigned>(cdiv(Vw, ST_T))),
                         256, 0, st>>>(G, 1, ldg, X, 1, H, Vw, H, BT, nullptr, dW, H, c0, 4);
@@ -341,7 +384,7 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
     }
     const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
     // dX[r][h] (+)= sum_v G[r][v] W[c0 + v][h]
-    Rec r_(rec, 6);
+    Rec r_(rec, 6, 2.0 * BT * static_cast<double>(Vw) * H);
     k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)), mt), 256, 0, st>>>(
         G, ldg, 1, W + static_cast<size_t>(c0) * H, 1, H, BT, H, Vw, dxpart, dX, H, 0, mode);
     FLKL_CUDA(cudaGetLastError());
@@ -400,7 +443,7 @@ const char* flkl_status_string(int s) {
     case FLKL_ERR_CUDA: return "CUDA runtime error";
     case FLKL_ERR_TIMEOUT: return "a device-side wait ran out of time";
     case FLKL_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
-    case FLKL_ERR_TOO_LARGE: return "sizes need more scratch than the fixed 64 MiB device scratch";
+    case FLKL_ERR_TOO_LARGE: return "sizes need more scratch than the fixed 128 MiB device scratch";
     default: return "unknown status";
   }
 }
@@ -451,7 +494,9 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
   {
     Rec r_(rec, 0);
     k_prepare<<<1, 1024, 0, st>>>(shift_labels, bt, static_cast<long long>(ignore_index),
-                                  reduction, v, temperature, reinterpret_cast<DevCtl*>(ws));
+                                  reduction, v, temperature, reinterpret_cast<DevCtl*>(ws),
+                                  reinterpret_cast<int*>(ws + P.off_cnt),
+                                  static_cast<int>(P.n_counters));
     FLKL_CUDA(cudaGetLastError());
   }
 
@@ -557,10 +602,11 @@ flkl_status flkl_forward_backward_profiled(
     int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
     float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
     void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
-    void** events, int* kinds, int capacity, int* n_launches) {
-  if (events == nullptr || kinds == nullptr || n_launches == nullptr || capacity < 0)
+    void** events, int* kinds, double* flops, int capacity, int* n_launches) {
+  if (events == nullptr || kinds == nullptr || flops == nullptr || n_launches == nullptr ||
+      capacity < 0)
     return FLKL_ERR_INVALID_ARG;
-  Recorder r{reinterpret_cast<cudaEvent_t*>(events), kinds, capacity, 0,
+  Recorder r{reinterpret_cast<cudaEvent_t*>(events), kinds, flops, capacity, 0,
              static_cast<cudaStream_t>(stream)};
   const flkl_status s = forward_backward_impl(
       X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype, temperature, eps, reduction,

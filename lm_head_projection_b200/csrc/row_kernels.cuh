@@ -18,11 +18,14 @@ struct DevCtl {
 
 // One block of 1024 threads.  Counts kept rows (a row is dropped when its
 // shift label equals ignore_index), derives the divisor of the reduction
-// (batchmean: N_valid, mean: N_valid * V, sum: 1) and resets the error flag.
+// (batchmean: N_valid, mean: N_valid * V, sum: 1), resets the error flag and
+// zeroes the tile counters of the call's persistent launches.
 __global__ void __launch_bounds__(1024) k_prepare(const int64_t* __restrict__ labels, int BT,
                                                   long long ignore_index, int reduction, int V,
-                                                  float temperature, DevCtl* ctl) {
+                                                  float temperature, DevCtl* ctl,
+                                                  int* counters, int n_counters) {
   __shared__ int warp_cnt[32];
+  for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
   int cnt = 0;
   if (labels == nullptr) {
     cnt = (threadIdx.x == 0) ? BT : 0;
@@ -47,34 +50,35 @@ __global__ void __launch_bounds__(1024) k_prepare(const int64_t* __restrict__ la
   }
 }
 
-// Merge of the per-tile statistics (m, s, A, B2, S) of each row, in tile
+// Merge of the per-group statistics (m, s, A, B2, S) of each row, in group
 // order, into lse2 = log2 sum 2^t and the row loss
 //   l_r = ln2 * B2 - A / T + ln2 * lse2 * S
 // (= sum_v q (log max(q,eps) - log p)).  Also the per-row coefficients of the
-// gradient pass.  Block: 8 warps x 32 rows; warp w merges tiles w, w+8, ...
-__global__ void __launch_bounds__(256) k_combine(const float* __restrict__ st, int n_tiles, int BT,
-                                                 const int64_t* __restrict__ labels,
-                                                 long long ignore_index, float invT,
-                                                 const DevCtl* __restrict__ ctl,
-                                                 float* __restrict__ lse2_out,
-                                                 float* __restrict__ coefS,
-                                                 float* __restrict__ coefQ,
-                                                 float* __restrict__ rowloss) {
-  __shared__ float part[8][5][32];
+// gradient pass.  Block: 32 warps x 32 rows; warp w merges groups w, w+32, ...
+// (loads coalesced over the 32 rows), then warp 0 merges the 32 partials in
+// warp order.
+constexpr int kCombineWarps = 32;
+__global__ void __launch_bounds__(32 * kCombineWarps)
+    k_combine(const float* __restrict__ st, int n_tiles, int BT, const int64_t* __restrict__ labels,
+              long long ignore_index, float invT, const DevCtl* __restrict__ ctl,
+              float* __restrict__ lse2_out, float* __restrict__ coefS, float* __restrict__ coefQ,
+              float* __restrict__ rowloss) {
+  __shared__ float part[kCombineWarps][5][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = blockIdx.x * 32 + lane;
   const size_t plane = static_cast<size_t>(n_tiles) * BT;
   float m = -INFINITY, s = 0.f, A = 0.f, B2 = 0.f, S = 0.f;
   if (row < BT) {
-    for (int t = w; t < n_tiles; t += 8) {
+#pragma unroll 4
+    for (int t = w; t < n_tiles; t += kCombineWarps) {
       const size_t o = static_cast<size_t>(t) * BT + row;
       const float tm = st[o], ts = st[o + plane];
-      const float nm = fmaxf(m, tm);
-      s = s * exp2f(m - nm) + ts * exp2f(tm - nm);
-      m = nm;
       A += st[o + 2 * plane];
       B2 += st[o + 3 * plane];
       S += st[o + 4 * plane];
+      const float nm = fmaxf(m, tm);
+      s = s * exp2f(m - nm) + ts * exp2f(tm - nm);
+      m = nm;
     }
   }
   part[w][0][lane] = m;
@@ -89,9 +93,9 @@ __global__ void __launch_bounds__(256) k_combine(const float* __restrict__ st, i
     A = part[0][2][lane];
     B2 = part[0][3][lane];
     S = part[0][4][lane];
-    for (int k = 1; k < 8; ++k) {
+    for (int k = 1; k < kCombineWarps; ++k) {
       const float tm = part[k][0][lane];
-      if (tm == -INFINITY) continue;  // warp k saw no tile of this row
+      if (tm == -INFINITY) continue;  // warp k saw no group of this row
       const float nm = fmaxf(m, tm);
       s = s * exp2f(m - nm) + part[k][1][lane] * exp2f(tm - nm);
       m = nm;

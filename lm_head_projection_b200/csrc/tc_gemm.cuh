@@ -1,258 +1,178 @@
-// Persistent warp-specialised tcgen05 GEMM for sm_100a with fused epilogues.
+// Persistent warp-specialised tcgen05 GEMM for sm_100a on CTA pairs, with
+// fused epilogues.
 //
 //   D[M,N] = A[M,K] * B[N,K]^T, bf16 operands, fp32 accumulation in TMEM.
 //
-// Roles (6 warps, one CTA per SM):
-//   warp 0      TMA producer: stages A and B tiles (SWIZZLE_128B) into a
-//               4-deep shared-memory ring, one mbarrier pair per stage;
-//   warp 1      MMA issuer: owns the TMEM allocation (512 columns = two
-//               128x256 fp32 accumulators) and issues tcgen05.mma from one
-//               thread; tcgen05.commit frees ring stages and publishes a
-//               finished accumulator;
-//   warps 2..5  epilogue: each warp reads its 32-lane quarter of the
-//               accumulator with tcgen05.ld (one thread = one output row) and
-//               runs the fused epilogue, while the MMA warp already fills the
-//               other accumulator with the next tile.
+// A cluster of two CTAs (on two SMs) computes one 256x256 output tile with
+// tcgen05.mma.cta_group::2: CTA r stages rows [128r, 128r+128) of the tile's
+// A block and rows [128r, 128r+128) of its B block, so each SM streams half
+// of B; the even CTA issues the MMAs, which read A and B from both CTAs'
+// shared memory and write rows [128r, 128r+128) of D into CTA r's TMEM.
+//
+// Roles (6 warps per CTA, one CTA per SM):
+//   warp 0      TMA producer (both CTAs): a 6-deep ring of 32 KiB stages;
+//               every copy signals the even CTA's `full` barrier;
+//   warp 1      TMEM owner (both CTAs, 512 columns = two 256-column fp32
+//               accumulators) and, in the even CTA, the MMA issuer;
+//               tcgen05.commit arrives on both CTAs' `empty` (stage free)
+//               and `tfull` (accumulator ready) barriers;
+//   warps 2..9  epilogue (both CTAs): warp w reads lane quarter w%4 of its
+//               CTA's accumulator, columns [128h, 128h+128) with h = (w-2)/4,
+//               with tcgen05.ld (one thread = one output row) while the MMA
+//               fills the other accumulator; the warps then arrive on the
+//               even CTA's `tempty` barrier.
 //
 // Operands may be K-major (rows of K contiguous) or MN-major (K rows of M or N
 // contiguous); both are loaded by plain 2-D TMA tile copies, never multicast.
-// Every wait is bounded (see mbar_wait); on a timeout the CTA drains its own
-// in-flight copies and MMAs, frees TMEM and returns.
+// Every wait is bounded (see mbar_wait); on a timeout the CTA stops, drains
+// its own in-flight copies and MMAs, frees TMEM and returns.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace flkl {
 
-constexpr int TC_BM = 128;
-constexpr int TC_BN = 256;
-constexpr int TC_BK = 64;
-constexpr int TC_STAGES = 4;
-constexpr int TC_THREADS = 192;
-constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;  // 16 KiB
-constexpr int TC_B_BYTES = TC_BN * TC_BK * 2;  // 32 KiB
+constexpr int TC_BM = 256;            // output tile rows (pair)
+constexpr int TC_BN = 256;            // output tile columns
+constexpr int TC_HM = 128;            // rows per CTA
+constexpr int TC_BK = 128;            // K depth of a ring stage (a multiple of 64)
+constexpr int TC_KSUB = TC_BK / 64;   // 128-byte swizzle atoms along K per stage
+constexpr int TC_STAGES = 3;
+constexpr int TC_PREFETCH_KB = 0;     // L2 prefetch distance of the producer, in k-blocks
+constexpr int TC_EPI_WARPS = 8;       // two per TMEM lane quarter
+constexpr int TC_EPI_COLS = 128;      // accumulator columns per epilogue warp
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
+constexpr int TC_A_BYTES = TC_HM * TC_BK * 2;  // 16 KiB: this CTA's A rows
+constexpr int TC_B_BYTES = TC_HM * TC_BK * 2;  // 16 KiB: this CTA's half of B
+constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_TMEM_COLS = 512;
-constexpr int TC_SMEM_BYTES = TC_STAGES * (TC_A_BYTES + TC_B_BYTES) + 256 + 1024;
+constexpr int TC_XPOSE_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 rows x 32 fp32
+constexpr int TC_SMEM_BYTES =
+    TC_STAGES * TC_STAGE_BYTES + TC_EPI_WARPS * TC_XPOSE_BYTES + 256 + 1024;
 
-struct TcGemmArgs {
-  int M, N, K;          // problem extent (rows of D, cols of D, reduction)
-  int m_tiles, n_tiles; // ceil(M/128), ceil(N/256)
-  int num_kb;           // ceil(K/64)
-  int m_fastest;        // tile order: 1 = consecutive tiles walk M
-  int a_m_off, a_k_off; // coordinate offsets added to A tile coordinates
-  int b_n_off, b_k_off; // coordinate offsets added to B tile coordinates
-  int* err_flag;
-  unsigned long long wait_limit_ns;
+static_assert(TC_SMEM_BYTES <= 232448, "dynamic shared memory above the sm_100 per-CTA limit");
+// Loads this CTA's 128 rows of one operand for one ring stage.  K-major:
+// TC_KSUB boxes {64 (K), 128}, 16 KiB apart.  MN-major: two boxes
+// {64 (MN), TC_BK (K)}, TC_BK * 128 bytes apart.
+__device__ __forceinline__ void tma_half_stage(const CUtensorMap* map, bool mn_major,
+                                               uint32_t bar_cluster, uint8_t* dst, int mn0,
+                                               int k0) {
+  if (!mn_major) {
+#pragma unroll
+    for (int s = 0; s < TC_KSUB; ++s)
+      tma_load_2d_pair(map, bar_cluster, dst + s * 16384, k0 + 64 * s, mn0);
+  } else {
+    tma_load_2d_pair(map, bar_cluster, dst, mn0, k0);
+    tma_load_2d_pair(map, bar_cluster, dst + TC_BK * 128, mn0 + 64, k0);
+  }
+}
+
+// L2 prefetch of the same boxes tma_half_stage would load.
+__device__ __forceinline__ void prefetch_half_stage(const CUtensorMap* map, bool mn_major, int mn0,
+                                                    int k0) {
+  if (!mn_major) {
+#pragma unroll
+    for (int s = 0; s < TC_KSUB; ++s) tma_prefetch_l2_2d(map, k0 + 64 * s, mn0);
+  } else {
+    tma_prefetch_l2_2d(map, mn0, k0);
+    tma_prefetch_l2_2d(map, mn0 + 64, k0);
+  }
+}
+
+// Descriptor of the k-th 16-deep slice of a stage (the same offsets are used
+// in both CTAs of the pair).
+__device__ __forceinline__ uint64_t stage_desc(uint32_t base, int k, bool mn_major) {
+  if (!mn_major) {
+    // 64-deep K sub-blocks of 128 rows x 128 B (16 KiB apart), 8-row atoms of
+    // 1024 B; K slice of 16 = +32 B inside the sub-block
+    return smem_desc_sw128(base + 16384u * (k >> 2) + 32u * (k & 3), 16u, 1024u);
+  } else {
+    // 64-wide MN blocks of TC_BK K-rows (TC_BK * 128 B apart = LBO), 8-row K
+    // groups of 1024 B (SBO); K slice of 16 rows = +2048 B
+    return smem_desc_sw128(base + 2048u * k, TC_BK * 128u, 1024u);
+  }
+}
+
+// The same descriptors as stage_desc, split for cheap issue: lower word =
+// lo_base + (stage address >> 4) + (k & 3) * s1 + (k >> 2) * s2, upper word hi.
+struct DescSteps {
+  uint32_t lo_base, hi, s1, s2;
 };
-
-__device__ __forceinline__ void tile_coords(const TcGemmArgs& g, int t, int& mb, int& nb) {
-  if (g.m_fastest) {
-    mb = t % g.m_tiles;
-    nb = t / g.m_tiles;
-  } else {
-    nb = t % g.n_tiles;
-    mb = t / g.n_tiles;
-  }
+__device__ __forceinline__ DescSteps desc_steps(bool mn_major) {
+  const uint64_t d = mn_major ? smem_desc_sw128(0, TC_BK * 128u, 1024u)
+                              : smem_desc_sw128(0, 16u, 1024u);
+  DescSteps r;
+  r.lo_base = static_cast<uint32_t>(d);
+  r.hi = static_cast<uint32_t>(d >> 32);
+  r.s1 = mn_major ? (2048u >> 4) : (32u >> 4);     // next 16-deep K slice
+  r.s2 = mn_major ? (8192u >> 4) : (16384u >> 4);  // next 64-deep K sub-block
+  return r;
 }
 
-// Loads one ring stage.  K-major operand tile: one box {64 (K), rows}.
-// MN-major operand tile: rows/64 boxes {64 (MN), 64 (K)}, 8 KiB apart.
-template <bool MN_MAJOR, int ROWS>
-__device__ __forceinline__ void tma_stage(const CUtensorMap* map, uint64_t* bar, uint8_t* dst,
-                                          int mn0, int k0) {
-  if constexpr (!MN_MAJOR) {
-    tma_load_2d(map, bar, dst, k0, mn0);
-  } else {
-#pragma unroll
-    for (int j = 0; j < ROWS / 64; ++j) tma_load_2d(map, bar, dst + j * 8192, mn0 + 64 * j, k0);
-  }
-}
-
-// Descriptor of the k-th 16-deep slice of a stage.
-template <bool MN_MAJOR>
-__device__ __forceinline__ uint64_t stage_desc(uint32_t base, int k) {
-  if constexpr (!MN_MAJOR) {
-    // rows of 128 B (64 bf16 of K), 8-row atoms of 1024 B; K slice = +32 B
-    return smem_desc_sw128(base + 32u * k, 16u, 1024u);
-  } else {
-    // 64-wide MN blocks of 64 K-rows (8 KiB apart = LBO), 8-row K groups of
-    // 1024 B (SBO); K slice of 16 rows = +2048 B
-    return smem_desc_sw128(base + 2048u * k, 8192u, 1024u);
-  }
-}
-
-template <class Epi, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(TC_THREADS, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcGemmArgs g, const typename Epi::Params ep) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * TC_B_BYTES);
-  uint64_t* full = bars;                   // [STAGES] TMA -> MMA
-  uint64_t* empty = bars + TC_STAGES;      // [STAGES] MMA -> TMA
-  uint64_t* tfull = bars + 2 * TC_STAGES;  // [2] MMA -> epilogue
-  uint64_t* tempty = tfull + 2;            // [2] epilogue -> MMA
-  uint64_t* drain = tempty + 2;            // MMA drain at exit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < TC_STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, TC_TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const WaitCtl wc{abort_flag, g.err_flag, g.wait_limit_ns};
-  const int num_tiles = g.m_tiles * g.n_tiles;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------ producer
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        int mb, nb;
-        tile_coords(g, t, mb, nb);
-        const int m0 = mb * TC_BM + g.a_m_off;
-        const int n0 = nb * TC_BN + g.b_n_off;
-        for (int kb = 0; kb < g.num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], TC_A_BYTES + TC_B_BYTES);
-          tma_stage<A_MN, TC_BM>(&tmA, &full[stage], sA + stage * TC_A_BYTES, m0,
-                                 kb * TC_BK + g.a_k_off);
-          tma_stage<B_MN, TC_BN>(&tmB, &full[stage], sB + stage * TC_B_BYTES, n0,
-                                 kb * TC_BK + g.b_k_off);
-          ++issued;
-          if (++stage == TC_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // Drain: the last min(issued, STAGES) copies must have landed before
-      // the CTA may exit (they always complete; the wait is still bounded).
-      int s = stage;
-      uint32_t ph = phase;
-      for (int i = 0; i < TC_STAGES && i < issued; ++i) {
-        if (--s < 0) {
-          s = TC_STAGES - 1;
-          ph ^= 1u;
-        }
-        const uint32_t addr = smem_u32(&full[s]);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(addr, ph)) {
-          if (globaltimer_ns() - t0 > g.wait_limit_ns) break;
-        }
-      }
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN, A_MN, B_MN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * TC_BN;
-        for (int kb = 0; kb < g.num_kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, wc)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + stage * TC_A_BYTES);
-          const uint32_t b_base = smem_u32(sB + stage * TC_B_BYTES);
-#pragma unroll
-          for (int k = 0; k < TC_BK / 16; ++k) {
-            tc_mma_f16(d_tmem, stage_desc<A_MN>(a_base, k), stage_desc<B_MN>(b_base, k), idesc,
-                       (kb | k) != 0 ? 1u : 0u);
-          }
-          tc_commit(&empty[stage]);
-          if (++stage == TC_STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (ok) tc_commit(&tfull[acc]);
-      }
-      // Drain every MMA this thread issued before TMEM is released.
-      tc_commit(drain);
-      const uint32_t addr = smem_u32(drain);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(addr, 0)) {
-        if (globaltimer_ns() - t0 > g.wait_limit_ns) break;
-      }
-    }
-    __syncwarp();
-  } else {
-    // -------------------------------------------------------- epilogue
-    const int quad = warp & 3;  // TMEM lane quarter this warp may access
-    int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], acc_phase, wc)) break;
-      __syncwarp();
-      tc_fence_after();
-      int mb, nb;
-      tile_coords(g, t, mb, nb);
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * TC_BN;
-      Epi::run(ep, g, taddr, mb, nb, quad, lane);
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-    }
-  }
-
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TC_TMEM_COLS);
+// Wait (bounded, no abort check) for phase `parity` of a local barrier; used
+// only on exit paths.
+__device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity,
+                                                unsigned long long limit_ns) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(addr, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) break;
   }
 }
 
 // ====================================================================
-// Epilogues.  `run` is called by each of the 4 epilogue warps for its
-// 32-row quarter; lane i owns row (mb*128 + quad*32 + i) of the tile.
+// Epilogues.  `run` is called by each epilogue warp for its 32 rows and 128
+// columns of the tile: lane i owns output row (row0 + quad*32 + i), columns
+// [n0, n0 + 128).  `prefetch` is called with the same coordinates just before
+// the warp waits for that tile's accumulator, so that the rows of Q the tile
+// needs are on their way to L2 while the MMAs run.
 
-// Pass 1: per (row, 256-column tile) softmax and KL statistics.
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(ptr)));
+}
+
+// Per-warp transpose through shared memory, so that a warp's global stores
+// cover whole 128-byte lines: lane r puts its row's 32 fp32 values (float4
+// slot j stored at slot j ^ (r & 7), bank-conflict free both ways); the warp
+// then reads them back four rows per instruction.
+__device__ __forceinline__ void xpose_put(float* buf, int lane, const float (&v)[32]) {
+  float4* b = reinterpret_cast<float4*>(buf) + lane * 8;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    b[j ^ (lane & 7)] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
+__device__ __forceinline__ float4 xpose_get(const float* buf, int r, int j) {
+  return reinterpret_cast<const float4*>(buf)[r * 8 + (j ^ (r & 7))];
+}
+__device__ __forceinline__ void st_global_bf16x4(void* dst, const float4& v) {
+  const uint32_t lo = pack_bf16x2(v.x, v.y), hi = pack_bf16x2(v.z, v.w);
+  asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(dst), "r"(lo), "r"(hi) : "memory");
+}
+
+// 32 bf16 of one row (four 16-byte loads), zero beyond `limit` or when !rv.
+__device__ __forceinline__ void load_chunk32(const __nv_bfloat16* rowp, bool rv, int col0,
+                                             int limit, uint4 (&u)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int cc = col0 + 8 * j;
+    u[j] = (rv && cc < limit) ? ld_nc_v4(rowp + cc) : make_uint4(0, 0, 0, 0);
+  }
+}
+// Same 32 bias values for every lane of the warp (one broadcast request).
+__device__ __forceinline__ void load_bias32(const __nv_bfloat16* bias, int col0, int V,
+                                            float (&bv)[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int cc = col0 + 8 * j;
+    uint4 u = make_uint4(0, 0, 0, 0);
+    if (bias != nullptr && cc < V) u = *reinterpret_cast<const uint4*>(bias + cc);
+    unpack8_bf16(u, bv + 8 * j);
+  }
+}
+
+// Pass 1: per (row, 128-column group) softmax and KL statistics.
 //   t = (acc + b) * log2(e)/T        (student logits in base-2 units)
-//   m = max t, s = sum 2^(t - m)     (online over the tile's 8 column groups)
+//   m = max t, s = sum 2^(t - m)     (online over the group's 32-column chunks)
 //   A = sum q z, B2 = sum q log2 max(q, eps), S = sum q
 struct EpiStats {
   struct Params {
@@ -261,32 +181,37 @@ struct EpiStats {
     int BT, V;
     float t_scale;  // log2(e) / T
     float eps;
-    float* st;      // [5][n_tiles][BT]
-    long long st_plane;  // n_tiles * BT
+    float* st;      // [5][n_groups][BT], n_groups = ceil(V/128)
+    long long st_plane;  // n_groups * BT
   };
-  __device__ __forceinline__ static void run(const Params& p, const TcGemmArgs&, uint32_t taddr,
-                                             int mb, int nb, int quad, int lane) {
-    const int row = mb * TC_BM + quad * 32 + lane;
+  __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
+                                                  int lane) {
+    const int row = row0 + quad * 32 + lane;
+    if (row < p.BT && n0 < p.V) {
+      const __nv_bfloat16* q = p.Q + static_cast<size_t>(row) * p.V + n0;
+      prefetch_l2(q);
+      if (n0 + 64 < p.V) prefetch_l2(q + 64);
+    }
+  }
+  __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
+                                             int quad, int lane, float* xbuf) {
+    const int row = row0 + quad * 32 + lane;
     const bool rv = row < p.BT;
-    const int n0 = nb * TC_BN;
+    if (n0 >= p.V) return;  // warp-uniform: this half of the tile is past V
     const __nv_bfloat16* qrow = p.Q + static_cast<size_t>(rv ? row : 0) * p.V;
     const float qmin = fmaxf(p.eps, 1.17549435e-38f);
     float m = -INFINITY, s = 0.f, A = 0.f, B2 = 0.f, S = 0.f;
+    uint4 qa[4], qb[4];
+    load_chunk32(qrow, rv, n0, p.V, qa);
 #pragma unroll 1
-    for (int c = 0; c < TC_BN / 32; ++c) {
+    for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
       const int col0 = n0 + c * 32;
       if (col0 >= p.V) break;  // warp-uniform
+      if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, col0 + 32, p.V, qb);
       float q[32], bv[32], z[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int cc = col0 + 8 * j;
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (rv && cc < p.V) u = ld_nc_v4(qrow + cc);
-        unpack8_bf16(u, q + 8 * j);
-        uint4 ub = make_uint4(0, 0, 0, 0);
-        if (p.bias != nullptr && cc < p.V) ub = ld_nc_v4(p.bias + cc);
-        unpack8_bf16(ub, bv + 8 * j);
-      }
+      for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+      load_bias32(p.bias, col0, p.V, bv);
       tmem_ld32(taddr + c * 32, z);
       float cm = -INFINITY;
 #pragma unroll
@@ -305,9 +230,11 @@ struct EpiStats {
       for (int i = 0; i < 32; ++i) acc += exp2f(z[i] - nm);
       s = acc;
       m = nm;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qa[j] = qb[j];
     }
     if (rv) {
-      const size_t o = static_cast<size_t>(nb) * p.BT + row;
+      const size_t o = static_cast<size_t>(n0 / TC_EPI_COLS) * p.BT + row;
       p.st[o] = m;
       p.st[o + p.st_plane] = s;
       p.st[o + 2 * p.st_plane] = A;
@@ -351,32 +278,37 @@ struct EpiGrad {
     const float* coefQ;  // [BT] 1 / (T D), 0 on dropped rows
     float* dbpart;       // [row groups of 32][V] or null
   };
-  __device__ __forceinline__ static void run(const Params& p, const TcGemmArgs&, uint32_t taddr,
-                                             int mb, int nb, int quad, int lane) {
-    const int row = mb * TC_BM + quad * 32 + lane;
-    const bool rv = row < p.BT;
-    const int n0 = nb * TC_BN;  // chunk-relative
+  __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
+                                                  int lane) {
+    const int row = row0 + quad * 32 + lane;
+    const int gc = p.c0 + n0;
+    if (row < p.BT && gc < p.V) {
+      const __nv_bfloat16* q = p.Q + static_cast<size_t>(row) * p.V + gc;
+      prefetch_l2(q);
+      if (gc + 64 < p.V) prefetch_l2(q + 64);
+    }
+  }
+  __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
+                                             int quad, int lane, float* xbuf) {
+    const int row = row0 + quad * 32 + lane;
+    const bool rv = row < p.BT;  // n0 is chunk-relative
+    if (p.c0 + n0 >= p.V) return;  // warp-uniform
     const __nv_bfloat16* qrow = p.Q + static_cast<size_t>(rv ? row : 0) * p.V;
-    __nv_bfloat16* grow = p.G + static_cast<size_t>(rv ? row : 0) * p.ldg;
     const float lse2 = rv ? p.lse2[row] : 0.f;
     const float cS = rv ? p.coefS[row] : 0.f;
     const float cQ = rv ? p.coefQ[row] : 0.f;
+    uint4 qa[4], qb[4];
+    load_chunk32(qrow, rv, p.c0 + n0, p.V, qa);
 #pragma unroll 1
-    for (int c = 0; c < TC_BN / 32; ++c) {
+    for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
       const int col0 = n0 + c * 32;
       const int gcol0 = p.c0 + col0;
       if (gcol0 >= p.V) break;  // warp-uniform
+      if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, gcol0 + 32, p.V, qb);
       float q[32], bv[32], z[32];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int cc = gcol0 + 8 * j;
-        uint4 u = make_uint4(0, 0, 0, 0);
-        if (rv && cc < p.V) u = ld_nc_v4(qrow + cc);
-        unpack8_bf16(u, q + 8 * j);
-        uint4 ub = make_uint4(0, 0, 0, 0);
-        if (p.bias != nullptr && cc < p.V) ub = ld_nc_v4(p.bias + cc);
-        unpack8_bf16(ub, bv + 8 * j);
-      }
+      for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+      load_bias32(p.bias, gcol0, p.V, bv);
       tmem_ld32(taddr + c * 32, z);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -385,24 +317,26 @@ struct EpiGrad {
         const float gv = cS * exp2f(t - lse2) - cQ * q[i];
         z[i] = ok ? gv : 0.f;
       }
-      if (rv) {
-        uint4* dst = reinterpret_cast<uint4*>(grow + col0);
+      // G -> staging: transpose so that each store covers 4 rows x 64 bytes
+      __syncwarp();
+      xpose_put(xbuf, lane, z);
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 u;
-          u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
-          u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
-          u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
-          u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
-          dst[j] = u;
-        }
+      for (int i = 0; i < 8; ++i) {
+        const int r = i * 4 + (lane >> 3), j = lane & 7;
+        const int grow_i = row0 + quad * 32 + r;
+        if (grow_i < p.BT)
+          st_global_bf16x4(p.G + static_cast<size_t>(grow_i) * p.ldg + col0 + 4 * j,
+                           xpose_get(xbuf, r, j));
       }
       if (p.dbpart != nullptr) {
         const float colsum = warp_transpose_sum32(z, lane);
         const int gc = gcol0 + lane;
         if (gc < p.V)
-          p.dbpart[static_cast<size_t>(mb * 4 + quad) * p.V + gc] = colsum;
+          p.dbpart[static_cast<size_t>(row0 / 32 + quad) * p.V + gc] = colsum;
       }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qa[j] = qb[j];
     }
   }
 };
@@ -417,36 +351,29 @@ struct EpiStoreRows {
     int row_off;    // first output row (chunk start)
     int out_fp32;
   };
-  __device__ __forceinline__ static void run(const Params& p, const TcGemmArgs&, uint32_t taddr,
-                                             int mb, int nb, int quad, int lane) {
-    const int r = mb * TC_BM + quad * 32 + lane;
-    const bool rv = r < p.rows;
-    const size_t orow = static_cast<size_t>(p.row_off + (rv ? r : 0)) * p.ld;
+  __device__ __forceinline__ static void prefetch(const Params&, int, int, int, int) {}
+  __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
+                                             int quad, int lane, float* xbuf) {
+    const int rbase = row0 + quad * 32;
 #pragma unroll 1
-    for (int c = 0; c < TC_BN / 32; ++c) {
-      const int col0 = nb * TC_BN + c * 32;
-      if (col0 >= p.cols) break;
+    for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
+      const int col0 = n0 + c * 32;
+      if (col0 >= p.cols) break;  // warp-uniform
       float v[32];
       tmem_ld32(taddr + c * 32, v);
-      if (!rv) continue;
-      if (p.out_fp32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + col0);
+      __syncwarp();
+      xpose_put(xbuf, lane, v);
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (col0 + 4 * j < p.cols)
-            dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow + col0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (col0 + 8 * j < p.cols) {
-            uint4 u;
-            u.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-            u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-            u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-            u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-            dst[j] = u;
-          }
+      for (int i = 0; i < 8; ++i) {
+        const int r = i * 4 + (lane >> 3), j = lane & 7;
+        const int col = col0 + 4 * j;
+        if (rbase + r < p.rows && col < p.cols) {
+          const size_t o = static_cast<size_t>(p.row_off + rbase + r) * p.ld + col;
+          const float4 val = xpose_get(xbuf, r, j);
+          if (p.out_fp32) *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = val;
+          else st_global_bf16x4(static_cast<__nv_bfloat16*>(p.out) + o, val);
+        }
       }
     }
   }
@@ -464,50 +391,393 @@ struct EpiAccumRows {
     int ld, rows, cols;
     int mode;
   };
-  __device__ __forceinline__ static void run(const Params& p, const TcGemmArgs&, uint32_t taddr,
-                                             int mb, int nb, int quad, int lane) {
-    const int r = mb * TC_BM + quad * 32 + lane;
-    const bool rv = r < p.rows;
-    const size_t orow = static_cast<size_t>(rv ? r : 0) * p.ld;
+  __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
+                                                  int lane) {
+    const int r = row0 + quad * 32 + lane;
+    if ((p.mode == 2 || p.mode == 3) && r < p.rows && n0 < p.cols) {
+      const float* q = p.part + static_cast<size_t>(r) * p.ld + n0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (n0 + 32 * j < p.cols) prefetch_l2(q + 32 * j);
+    }
+  }
+  __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
+                                             int quad, int lane, float* xbuf) {
+    const int rbase = row0 + quad * 32;
 #pragma unroll 1
-    for (int c = 0; c < TC_BN / 32; ++c) {
-      const int col0 = nb * TC_BN + c * 32;
-      if (col0 >= p.cols) break;
+    for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
+      const int col0 = n0 + c * 32;
+      if (col0 >= p.cols) break;  // warp-uniform
       float v[32];
       tmem_ld32(taddr + c * 32, v);
-      if (!rv) continue;
-      float4* pp = reinterpret_cast<float4*>(p.part + orow + col0);
-      if (p.mode == 2 || p.mode == 3) {
+      __syncwarp();
+      xpose_put(xbuf, lane, v);
+      __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (col0 + 4 * j < p.cols) {
-            const float4 o = pp[j];
-            v[4 * j] += o.x;
-            v[4 * j + 1] += o.y;
-            v[4 * j + 2] += o.z;
-            v[4 * j + 3] += o.w;
+      for (int i = 0; i < 8; ++i) {
+        const int r = i * 4 + (lane >> 3), j = lane & 7;
+        const int col = col0 + 4 * j;
+        if (rbase + r < p.rows && col < p.cols) {
+          const size_t o = static_cast<size_t>(rbase + r) * p.ld + col;
+          float4 val = xpose_get(xbuf, r, j);
+          if (p.mode == 2 || p.mode == 3) {
+            const float4 prev = *reinterpret_cast<const float4*>(p.part + o);
+            val.x += prev.x;
+            val.y += prev.y;
+            val.z += prev.z;
+            val.w += prev.w;
           }
-      }
-      if (p.mode == 1 || p.mode == 2) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (col0 + 4 * j < p.cols)
-            pp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + orow + col0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (col0 + 8 * j < p.cols) {
-            uint4 u;
-            u.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
-            u.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
-            u.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
-            u.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
-            dst[j] = u;
-          }
+          if (p.mode == 1 || p.mode == 2) *reinterpret_cast<float4*>(p.part + o) = val;
+          else st_global_bf16x4(p.out + o, val);
+        }
       }
     }
   }
 };
+
+
+// ====================================================================
+// Launch descriptor: up to three GEMM problems served by one persistent
+// launch.  Their tiles form one sequence [problem 0 tiles, problem 1 tiles,
+// ...]; CTA pairs claim tiles in that order from a global counter, so the
+// longest tiles (placed first) start first and the shortest fill the end.
+
+enum TcKind : int {
+  KIND_STATS = 0,  // z tile -> softmax/KL statistics      A = X (K-major), B = W (K-major)
+  KIND_GRAD = 1,   // z tile -> G staging (+ db partials)   A = X (K-major), B = W (K-major)
+  KIND_DW = 2,     // dW rows = G^T X                       A = G (MN-major), B = X (MN-major)
+  KIND_DX = 3      // dX (+)= G W                           A = G (K-major), B = W (MN-major)
+};
+__host__ __device__ constexpr bool kind_a_mn(int k) { return k == KIND_DW; }
+__host__ __device__ constexpr bool kind_b_mn(int k) { return k == KIND_DW || k == KIND_DX; }
+
+constexpr int TC_MAX_PROBLEMS = 3;
+constexpr int TC_SLOTS = 4;  // depth of the tile-id ring
+
+struct TcProblem {
+  int kind;
+  int m_tiles, n_tiles;   // 256 x 256 tiles
+  int num_kb;             // K / 64, rounded up
+  int m_fastest;          // tile order inside the problem
+  int a_m_off, a_k_off;   // offsets added to A tile coordinates
+  int b_n_off, b_k_off;   // offsets added to B tile coordinates
+  int tile_begin;         // first tile of the problem in the launch sequence
+};
+
+struct TcMaps {
+  CUtensorMap m[2 * TC_MAX_PROBLEMS];  // A and B of each problem
+};
+
+struct TcLaunch {
+  int nprob;
+  int total_tiles;
+  int mix;  // interleave problems 1 and 2 (see find_problem)
+  TcProblem prob[TC_MAX_PROBLEMS];
+  int* counter;  // tile counter of this launch, 0 at launch
+  int* err_flag;
+  unsigned long long wait_limit_ns;
+  EpiStats::Params stats;
+  EpiGrad::Params grad;
+  EpiStoreRows::Params dw;
+  EpiAccumRows::Params dx;
+};
+
+// Problem and local tile index of sequence position t.  Problem 0 occupies
+// the first tiles; when L.mix is set, problems 1 and 2 are interleaved in
+// proportion to their tile counts over the rest of the sequence (so that
+// compute-heavy and store-heavy tiles run side by side), otherwise they
+// follow one another.
+__device__ __forceinline__ int find_problem(const TcLaunch& L, int t, int& local) {
+  if (L.nprob == 1 || t < L.prob[1].tile_begin) {
+    local = t;
+    return 0;
+  }
+  const int j = t - L.prob[1].tile_begin;
+  if (L.mix && L.nprob == 3) {
+    const long long n1 = L.prob[1].m_tiles * static_cast<long long>(L.prob[1].n_tiles);
+    const long long n = L.total_tiles - L.prob[1].tile_begin;
+    const long long c_j = (static_cast<long long>(j) * n1) / n;        // problem-1 tiles before j
+    const long long c_j1 = (static_cast<long long>(j + 1) * n1) / n;
+    if (c_j1 > c_j) {
+      local = static_cast<int>(c_j);
+      return 1;
+    }
+    local = static_cast<int>(j - c_j);
+    return 2;
+  }
+  if (L.nprob == 3 && t >= L.prob[2].tile_begin) {
+    local = t - L.prob[2].tile_begin;
+    return 2;
+  }
+  local = j;
+  return 1;
+}
+
+__device__ __forceinline__ void problem_tile(const TcProblem& P, int local, int& mb, int& nb) {
+  if (P.m_fastest) {
+    mb = local % P.m_tiles;
+    nb = local / P.m_tiles;
+  } else {
+    nb = local % P.n_tiles;
+    mb = local / P.n_tiles;
+  }
+}
+
+template <class F>
+__device__ __forceinline__ void dispatch_epilogue(const TcLaunch& L, int kind, F&& f) {
+  switch (kind) {
+    case KIND_STATS: f(EpiStats{}, L.stats); break;
+    case KIND_GRAD: f(EpiGrad{}, L.grad); break;
+    case KIND_DW: f(EpiStoreRows{}, L.dw); break;
+    default: f(EpiAccumRows{}, L.dx); break;
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
+    tc_group_kernel(const __grid_constant__ TcMaps maps, const __grid_constant__ TcLaunch L) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
+  float* xpose = reinterpret_cast<float*>(sB + TC_STAGES * TC_B_BYTES);  // [EPI_WARPS][32*32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * TC_B_BYTES +
+                                               TC_EPI_WARPS * TC_XPOSE_BYTES);
+  uint64_t* full = bars;                       // [STAGES] TMA -> MMA (even CTA's are used)
+  uint64_t* empty = full + TC_STAGES;          // [STAGES] MMA -> TMA (each CTA)
+  uint64_t* tfull = empty + TC_STAGES;         // [2] MMA -> epilogue (each CTA)
+  uint64_t* tempty = tfull + 2;                // [2] epilogues -> MMA (even CTA's are used)
+  uint64_t* drain = tempty + 2;                // MMA drain at exit (even CTA)
+  uint64_t* tid_full = drain + 1;              // [SLOTS] tile id published (each CTA)
+  uint64_t* tid_empty = tid_full + TC_SLOTS;   // [SLOTS] tile id read (even CTA's are used)
+  int* tile_id = reinterpret_cast<int*>(tid_empty + TC_SLOTS);  // [SLOTS]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_id + TC_SLOTS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_cta_rank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < TC_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * TC_EPI_WARPS);  // every epilogue warp of both CTAs
+    }
+    mbar_init(drain, 1);
+    for (int k = 0; k < TC_SLOTS; ++k) {
+      mbar_init(&tid_full[k], 1);
+      // readers of a tile id: the MMA thread, the odd CTA's producer, every epilogue warp
+      mbar_init(&tid_empty[k], 2 + 2 * TC_EPI_WARPS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < 2 * L.nprob; ++i) tma_prefetch_desc(&maps.m[i]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, TC_TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers are initialised before anything targets them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, L.err_flag, L.wait_limit_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------ producer
+      int slot = 0, stage = 0, issued = 0;
+      uint32_t sph = 0, phase = 0;
+      bool ok = true;
+      // the even CTA claims one tile ahead, so the atomic's round trip
+      // overlaps the loads of the current tile
+      int claimed = leader ? atomicAdd(L.counter, 1) : 0;
+      while (ok) {
+        int t;
+        if (leader) {
+          // publish the claimed tile to both CTAs of the pair
+          if (!mbar_wait(&tid_empty[slot], sph ^ 1u, wc)) break;
+          t = claimed;
+          if (t < L.total_tiles) claimed = atomicAdd(L.counter, 1);
+          tile_id[slot] = t;
+          st_shared_cluster_u32(mapa_shared(smem_u32(&tile_id[slot]), 1),
+                                static_cast<uint32_t>(t));
+          mbar_arrive(&tid_full[slot]);
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tid_full[slot]), 1));
+        } else {
+          if (!mbar_wait_cluster(&tid_full[slot], sph, wc)) break;
+          t = tile_id[slot];
+          mbar_arrive_cluster(mapa_shared(smem_u32(&tid_empty[slot]), 0));
+        }
+        if (++slot == TC_SLOTS) {
+          slot = 0;
+          sph ^= 1u;
+        }
+        if (t >= L.total_tiles) break;
+        int local;
+        const int pi = find_problem(L, t, local);
+        const TcProblem& P = L.prob[pi];
+        const bool a_mn = kind_a_mn(P.kind), b_mn = kind_b_mn(P.kind);
+        int mb, nb;
+        problem_tile(P, local, mb, nb);
+        const int m0 = mb * TC_BM + static_cast<int>(rank) * TC_HM + P.a_m_off;
+        const int n0 = nb * TC_BN + static_cast<int>(rank) * TC_HM + P.b_n_off;
+        const CUtensorMap* mA = &maps.m[2 * pi];
+        const CUtensorMap* mB = &maps.m[2 * pi + 1];
+        for (int kb = 0; kb < P.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * TC_STAGE_BYTES);
+          tma_half_stage(mA, a_mn, fbar, sA + stage * TC_A_BYTES, m0, kb * TC_BK + P.a_k_off);
+          tma_half_stage(mB, b_mn, fbar, sB + stage * TC_B_BYTES, n0, kb * TC_BK + P.b_k_off);
+          if (TC_PREFETCH_KB > 0 && kb + TC_PREFETCH_KB < P.num_kb) {
+            // keep the L2 a few k-blocks ahead of the copies (HBM misses become L2 hits)
+            const int kp = (kb + TC_PREFETCH_KB) * TC_BK;
+            prefetch_half_stage(mA, a_mn, m0, kp + P.a_k_off);
+            prefetch_half_stage(mB, b_mn, n0, kp + P.b_k_off);
+          }
+          ++issued;
+          if (++stage == TC_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: every stage this CTA filled must have been consumed by the
+      // pair's MMAs (their commit arrives on `empty`) before the CTA exits.
+      int s = stage;
+      uint32_t ph = phase;
+      for (int i = 0; i < TC_STAGES && i < issued; ++i) {
+        if (--s < 0) {
+          s = TC_STAGES - 1;
+          ph ^= 1u;
+        }
+        mbar_drain_wait(&empty[s], ph, L.wait_limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------ MMA issuer
+      int slot = 0, stage = 0, it = 0;
+      uint32_t sph = 0, phase = 0;
+      bool ok = true;
+      while (ok) {
+        if (!mbar_wait(&tid_full[slot], sph, wc)) break;
+        const int t = tile_id[slot];
+        mbar_arrive(&tid_empty[slot]);
+        if (++slot == TC_SLOTS) {
+          slot = 0;
+          sph ^= 1u;
+        }
+        if (t >= L.total_tiles) break;
+        int local;
+        const TcProblem& P = L.prob[find_problem(L, t, local)];
+        const bool a_mn = kind_a_mn(P.kind), b_mn = kind_b_mn(P.kind);
+        const uint32_t idesc = idesc_bf16_f32(TC_BM, TC_BN, a_mn, b_mn);
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, wc)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * TC_BN;
+        // Descriptors of this tile: a constant upper word (SBO, version,
+        // swizzle) and a lower word (LBO | start address >> 4) that only moves
+        // by fixed steps between K slices and stages (see stage_desc).
+        const DescSteps da = desc_steps(a_mn), db = desc_steps(b_mn);
+        const uint32_t a_lo0 = da.lo_base + (smem_u32(sA) >> 4);
+        const uint32_t b_lo0 = db.lo_base + (smem_u32(sB) >> 4);
+        for (int kb = 0; kb < P.num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_lo = a_lo0 + stage * (TC_A_BYTES >> 4);
+          const uint32_t b_lo = b_lo0 + stage * (TC_B_BYTES >> 4);
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k) {
+            const uint64_t adesc =
+                (static_cast<uint64_t>(da.hi) << 32) | (a_lo + (k & 3) * da.s1 + (k >> 2) * da.s2);
+            const uint64_t bdesc =
+                (static_cast<uint64_t>(db.hi) << 32) | (b_lo + (k & 3) * db.s1 + (k >> 2) * db.s2);
+            tc_mma_pair_f16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == TC_STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit_pair(&tfull[acc], 0x3);
+        ++it;
+      }
+      // Drain every MMA this thread issued before TMEM is released.
+      tc_commit_pair(drain, 0x1);
+      mbar_drain_wait(drain, 0, L.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------- epilogue
+    const int quad = warp & 3;         // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // which 128 accumulator columns
+    const int rbase = static_cast<int>(rank) * TC_HM;
+    float* xbuf = xpose + (warp - 2) * (TC_XPOSE_BYTES / 4);
+    int slot = 0, it = 0;
+    uint32_t sph = 0;
+    while (true) {
+      if (!mbar_wait_cluster(&tid_full[slot], sph, wc)) break;
+      const int t = tile_id[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tid_empty[slot]), 0));
+      if (++slot == TC_SLOTS) {
+        slot = 0;
+        sph ^= 1u;
+      }
+      if (t >= L.total_tiles) break;
+      int local;
+      const TcProblem& P = L.prob[find_problem(L, t, local)];
+      int mb, nb;
+      problem_tile(P, local, mb, nb);
+      const int row0 = mb * TC_BM + rbase;
+      const int n0 = nb * TC_BN + half * TC_EPI_COLS;
+      dispatch_epilogue(L, P.kind, [&](auto epi, const auto& prm) {
+        decltype(epi)::prefetch(prm, row0, n0, quad, lane);
+      });
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull[acc], acc_phase, wc)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * TC_BN +
+                             half * TC_EPI_COLS;
+      dispatch_epilogue(L, P.kind, [&](auto epi, const auto& prm) {
+        decltype(epi)::run(prm, taddr, row0, n0, quad, lane, xbuf);
+      });
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      ++it;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA frees TMEM or leaves while the pair still works
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TC_TMEM_COLS);
+  }
+}
 
 }  // namespace flkl

@@ -55,16 +55,16 @@ def test_workspace_size_rules():
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_workspace_has_no_bt_by_v_buffer(name):
-    """The staged gradient block is at most BT x V/8 (plus tile rounding), and
-    the logits are never stored: the whole workspace stays well below one
-    BT x V array of the input dtype."""
+    """The two staged gradient blocks are at most BT x V/8 each (plus tile
+    rounding), and the logits are never stored: the whole workspace stays
+    below half of one BT x V array of the input dtype."""
     w = WORKLOADS[name]
     elem = 4 if w.dtype == "fp32" else 2
     need = pkg.flkl_workspace_size(w.BT, w.H, w.V, 0 if w.dtype == "fp32" else 1, w.compute_dW,
                                    w.compute_db)
     full = w.BT * w.V * elem
     if w.V >= 8 * 256:
-        assert need < 0.35 * full, (need, full)
+        assert need < 0.5 * full, (need, full)
 
 
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(),

@@ -219,7 +219,7 @@ def test_no_bt_by_v_allocation_at_full_size():
                          workspace=r["workspace"])
     torch.cuda.synchronize()
     assert torch.cuda.max_memory_allocated(dev) - base == 0
-    assert r["workspace"].numel() < w.BT * w.V * 2 // 4
+    assert r["workspace"].numel() < w.BT * w.V * 2 // 2
 
 
 def test_profiled_entry_records_every_launch_and_matches():
@@ -238,17 +238,21 @@ def test_profiled_entry_records_every_launch_and_matches():
     for e in events:
         e.record(stream)
     p = lambda t: None if t is None else t.data_ptr()
-    st, kinds, n = pkg.flkl_forward_backward_profiled(
+    st, kinds, flops, n = pkg.flkl_forward_backward_profiled(
         p(g["X"]), p(g["W"]), p(g["b"]), p(g["Q"]), None, -100, w.BT, w.H, w.V, 1, 1.0, 1e-10, 0,
         1, 1, 1, p(out["loss"]), p(out["dX"]), p(out["dW"]), p(out["db"]), p(ws), ws.numel(),
         stream.cuda_stream, events, cap)
     torch.cuda.synchronize()
     assert st == 0 and n == len(kinds)
     names = [pkg.LAUNCH_KINDS[k] for k in kinds]
-    nchunks = names.count("grad")
+    nchunks = names.count("chunk")
     assert nchunks >= 2
-    assert names == (["prepare", "stats", "combine", "loss"] + ["grad", "dW", "dX"] * nchunks
+    assert names == (["prepare", "stats", "combine", "loss", "grad"] + ["chunk"] * nchunks
                      + ["db"])
+    # every GEMM FLOP of the call is attributed once: stats, pass 2, dX and dW
+    gemm = 2.0 * w.BT * w.H * w.V
+    assert abs(sum(flops) - 4 * gemm) <= 1e-6 * gemm
+    assert flops[0] == 0.0 and flops[-1] == 0.0
     for i in range(n):
         assert events[2 * i].elapsed_time(events[2 * i + 1]) >= 0.0
     for k in ("loss", "dX", "dW", "db"):
