@@ -54,6 +54,39 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources the GEMM kernel is built from."""
+    import hashlib
+
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lm_head_projection_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def dram_traffic(workload: str, launch_kind: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+    `launch_kind` for `workload`, from the committed ncu summary, or None when
+    there is none or the kernel sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if line.startswith("- ") and ":" in line:
+                k, v = line[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    v = vals.get(f"dram_bytes_per_launch_{launch_kind}")
+    return float(v) if v else None
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -131,6 +164,18 @@ def dist_setup(n_gpus):
         raise SystemExit(f"--gpus {n_gpus} needs {n_gpus} ranks (WORLD_SIZE={world}); launch "
                          "with python -m torch.distributed.run --nproc-per-node N")
     return world, rank, local
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The maximum of `value` over all ranks (a no-op without a process
+    group): a multi-GPU time is the slowest rank's time."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def oracle_sample(w, rows, seed=123):
@@ -226,11 +271,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
     status = pkg.flkl_device_status(ws.data_ptr(), stream.cuda_stream)
     if status != 0:
         raise pkg.FlklError(status, "device status after the timed region")
@@ -265,7 +306,8 @@ def run_ours(args):
     if dom_flops > 0:
         achieved = dom_flops / (dom_ms * 1e-3) / 1e12  # = flops per launch / avg launch time
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_sust,
-                    "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4), "traffic": None,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
+                    "traffic": dram_traffic(w.name, dominant),
                     "kernel": f"tc_group_kernel ({dominant} launches)",
                     "flops_per_launch": dom_flops / dom_n,
                     "avg_launch_ms": round(dom_ms / dom_n, 4),
@@ -326,11 +368,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e = {"value": round(tokens / (e2e_ms / args.steps * 1e-3), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
 

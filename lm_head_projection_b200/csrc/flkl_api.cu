@@ -139,6 +139,26 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
+// bf16 3-D "blocked" tensor map over a row-major [outer][inner] matrix whose
+// blocked extent is a multiple of 64: dims {64, rows of the other extent,
+// blocked extent / 64}, the third dimension stepping 128 bytes.  K-major
+// operands block K (box {64, 128, TC_KSUB}); MN-major operands block MN
+// (box {64, TC_BK, 2}).  Returns false when the driver refuses the layout.
+bool make_blocked_map(CUtensorMap* m, const void* base, uint64_t blocked_extent,
+                      uint64_t other_extent, uint64_t pitch, bool mn_major) {
+  auto fn = encode_fn();
+  if (fn == nullptr || blocked_extent % 64 != 0) return false;
+  cuuint64_t dims[3] = {64, other_extent, blocked_extent / 64};
+  cuuint64_t strides[2] = {pitch * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(mn_major ? TC_BK : TC_HM),
+                       static_cast<cuuint32_t>(mn_major ? 2 : TC_KSUB)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_group(const TcMaps& maps, const TcLaunch& L, cudaStream_t st) {
   static bool attr_done[kMaxDevices] = {};
   int dev = 0;
@@ -156,10 +176,30 @@ cudaError_t launch_group(const TcMaps& maps, const TcLaunch& L, cudaStream_t st)
   return cudaGetLastError();
 }
 
+// One GEMM operand: its tensor map and whether the map is the 3-D blocked
+// form (one copy per half-stage) or the plain 2-D form.
+struct Operand {
+  CUtensorMap map;
+  int blocked;
+};
+
+// Operand over a row-major [outer][inner] bf16 matrix (pitch in elements),
+// K-major (inner = K) or MN-major (inner = M or N).  Uses the blocked 3-D map
+// when the inner extent is a multiple of 64, else the 2-D map.
+bool make_operand(Operand* o, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch,
+                  bool mn_major) {
+  if (make_blocked_map(&o->map, base, inner, outer, pitch, mn_major)) {
+    o->blocked = 1;
+    return true;
+  }
+  o->blocked = 0;
+  return make_map(&o->map, base, inner, outer, pitch, mn_major ? TC_BK : TC_HM);
+}
+
 // Appends a problem D[M,N] (K deep) of `kind` to launch L; A and B are its
-// tensor maps.  Returns false when L is full.
+// operands.  Returns false when L is full.
 bool add_problem(TcLaunch& L, TcMaps& maps, int kind, long long M, long long N, long long K,
-                 int m_fastest, const CUtensorMap& A, const CUtensorMap& B, int a_k_off = 0,
+                 int m_fastest, const Operand& A, const Operand& B, int a_k_off = 0,
                  int b_n_off = 0, int b_k_off = 0) {
   if (L.nprob >= TC_MAX_PROBLEMS) return false;
   TcProblem& P = L.prob[L.nprob];
@@ -173,8 +213,10 @@ bool add_problem(TcLaunch& L, TcMaps& maps, int kind, long long M, long long N, 
   P.b_n_off = b_n_off;
   P.b_k_off = b_k_off;
   P.tile_begin = L.total_tiles;
-  maps.m[2 * L.nprob] = A;
-  maps.m[2 * L.nprob + 1] = B;
+  P.a_blocked = A.blocked;
+  P.b_blocked = B.blocked;
+  maps.m[2 * L.nprob] = A.map;
+  maps.m[2 * L.nprob + 1] = B.map;
   L.total_tiles += P.m_tiles * P.n_tiles;
   ++L.nprob;
   return true;
@@ -241,9 +283,9 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
   const float t_scale = LOG2E / T;
   const int ldg = static_cast<int>(P.Vc);
 
-  CUtensorMap mX_k, mW_k, mX_mn, mW_mn;
-  if (!make_map(&mX_k, X, H, BT, H, TC_HM) || !make_map(&mW_k, W, H, V, H, TC_HM) ||
-      !make_map(&mX_mn, X, H, BT, H, TC_BK) || !make_map(&mW_mn, W, H, V, H, TC_BK))
+  Operand mX_k, mW_k, mX_mn, mW_mn;
+  if (!make_operand(&mX_k, X, H, BT, H, false) || !make_operand(&mW_k, W, H, V, H, false) ||
+      !make_operand(&mX_mn, X, H, BT, H, true) || !make_operand(&mW_mn, W, H, V, H, true))
     return FLKL_ERR_CUDA;
 
   auto new_launch = [&](int counter_index) {
@@ -300,8 +342,8 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
   for (long long c = 0; c < P.nchunks; ++c) {
     const int c0 = chunk_c0(c), Vw = chunk_w(c);
     __nv_bfloat16* G = Gbuf[c & 1];
-    CUtensorMap mG_k, mG_mn;
-    if (!make_map(&mG_k, G, Vw, BT, ldg, TC_HM) || !make_map(&mG_mn, G, Vw, BT, ldg, TC_BK))
+    Operand mG_k, mG_mn;
+    if (!make_operand(&mG_k, G, Vw, BT, ldg, false) || !make_operand(&mG_mn, G, Vw, BT, ldg, true))
       return FLKL_ERR_CUDA;
     TcLaunch L = new_launch(static_cast<int>(2 + c));
     TcMaps maps{};
@@ -311,7 +353,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     if (c + 1 < P.nchunks) add_grad(L, maps, c + 1);
     if (compute_dW) {
       L.dw = EpiStoreRows::Params{dW, H, Vw, H, c0, accum_fp32};
-      add_problem(L, maps, KIND_DW, Vw, H, BT, 0, mG_mn, mX_mn);
+      add_problem(L, maps, KIND_DW, Vw, H, BT, 1, mG_mn, mX_mn);
     }
     L.mix = 0;  // problems in sequence (interleaving pass-2 and dW tiles measured slower)
     double f = 2.0 * BT * static_cast<double>(Vw) * H * (1 + (compute_dW ? 1 : 0));

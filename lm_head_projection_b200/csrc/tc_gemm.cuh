@@ -46,17 +46,23 @@ constexpr int TC_A_BYTES = TC_HM * TC_BK * 2;  // 16 KiB: this CTA's A rows
 constexpr int TC_B_BYTES = TC_HM * TC_BK * 2;  // 16 KiB: this CTA's half of B
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_TMEM_COLS = 512;
-constexpr int TC_XPOSE_BYTES = 32 * 32 * 4;  // per epilogue warp: 32 rows x 32 fp32
-constexpr int TC_SMEM_BYTES =
-    TC_STAGES * TC_STAGE_BYTES + TC_EPI_WARPS * TC_XPOSE_BYTES + 256 + 1024;
+constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 256 + 1024;
 
 static_assert(TC_SMEM_BYTES <= 232448, "dynamic shared memory above the sm_100 per-CTA limit");
 // Loads this CTA's 128 rows of one operand for one ring stage.  K-major:
 // TC_KSUB boxes {64 (K), 128}, 16 KiB apart.  MN-major: two boxes
-// {64 (MN), TC_BK (K)}, TC_BK * 128 bytes apart.
-__device__ __forceinline__ void tma_half_stage(const CUtensorMap* map, bool mn_major,
+// {64 (MN), TC_BK (K)}, TC_BK * 128 bytes apart.  When the blocked extent is
+// a multiple of 64, a 3-D map whose third dimension steps 64 elements (128
+// bytes) along the blocked extent fetches the same bytes in one copy.
+__device__ __forceinline__ void tma_half_stage(const CUtensorMap* map, bool mn_major, bool blocked,
                                                uint32_t bar_cluster, uint8_t* dst, int mn0,
                                                int k0) {
+  if (blocked) {
+    // 3-D map {64, outer, blocks of 64}: the whole half-stage in one copy
+    if (!mn_major) tma_load_3d_pair(map, bar_cluster, dst, 0, mn0, k0 >> 6);
+    else tma_load_3d_pair(map, bar_cluster, dst, 0, k0, mn0 >> 6);
+    return;
+  }
   if (!mn_major) {
 #pragma unroll
     for (int s = 0; s < TC_KSUB; ++s)
@@ -131,23 +137,6 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(ptr)));
 }
 
-// Per-warp transpose through shared memory, so that a warp's global stores
-// cover whole 128-byte lines: lane r puts its row's 32 fp32 values (float4
-// slot j stored at slot j ^ (r & 7), bank-conflict free both ways); the warp
-// then reads them back four rows per instruction.
-__device__ __forceinline__ void xpose_put(float* buf, int lane, const float (&v)[32]) {
-  float4* b = reinterpret_cast<float4*>(buf) + lane * 8;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    b[j ^ (lane & 7)] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-}
-__device__ __forceinline__ float4 xpose_get(const float* buf, int r, int j) {
-  return reinterpret_cast<const float4*>(buf)[r * 8 + (j ^ (r & 7))];
-}
-__device__ __forceinline__ void st_global_bf16x4(void* dst, const float4& v) {
-  const uint32_t lo = pack_bf16x2(v.x, v.y), hi = pack_bf16x2(v.z, v.w);
-  asm volatile("st.global.v2.b32 [%0], {%1, %2};" ::"l"(dst), "r"(lo), "r"(hi) : "memory");
-}
 
 // 32 bf16 of one row (four 16-byte loads), zero beyond `limit` or when !rv.
 __device__ __forceinline__ void load_chunk32(const __nv_bfloat16* rowp, bool rv, int col0,
@@ -194,7 +183,7 @@ struct EpiStats {
     }
   }
   __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
-                                             int quad, int lane, float* xbuf) {
+                                             int quad, int lane) {
     const int row = row0 + quad * 32 + lane;
     const bool rv = row < p.BT;
     if (n0 >= p.V) return;  // warp-uniform: this half of the tile is past V
@@ -289,7 +278,7 @@ struct EpiGrad {
     }
   }
   __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
-                                             int quad, int lane, float* xbuf) {
+                                             int quad, int lane) {
     const int row = row0 + quad * 32 + lane;
     const bool rv = row < p.BT;  // n0 is chunk-relative
     if (p.c0 + n0 >= p.V) return;  // warp-uniform
@@ -317,17 +306,18 @@ struct EpiGrad {
         const float gv = cS * exp2f(t - lse2) - cQ * q[i];
         z[i] = ok ? gv : 0.f;
       }
-      // G -> staging: transpose so that each store covers 4 rows x 64 bytes
-      __syncwarp();
-      xpose_put(xbuf, lane, z);
-      __syncwarp();
+      if (rv) {
+        // this row's 32 gradients of the chunk: two full 32-byte sectors
+        uint4* dst = reinterpret_cast<uint4*>(p.G + static_cast<size_t>(row) * p.ldg + col0);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = i * 4 + (lane >> 3), j = lane & 7;
-        const int grow_i = row0 + quad * 32 + r;
-        if (grow_i < p.BT)
-          st_global_bf16x4(p.G + static_cast<size_t>(grow_i) * p.ldg + col0 + 4 * j,
-                           xpose_get(xbuf, r, j));
+        for (int j = 0; j < 4; ++j) {
+          uint4 u;
+          u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
+          u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
+          u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
+          u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
+          dst[j] = u;
+        }
       }
       if (p.dbpart != nullptr) {
         const float colsum = warp_transpose_sum32(z, lane);
@@ -342,6 +332,12 @@ struct EpiGrad {
 };
 
 // dW rows of one chunk: out[c0 + m][n] = acc, fp32 or bf16.
+// The store epilogues read the accumulator in the 16-lane fragment layout
+// (tmem_ld16x32): for each 32-column chunk and each 16-row half of the warp's
+// 32 rows, the threads of a quad hold 8 consecutive columns of a row, so one
+// warp store of 8-byte pairs writes 8 rows x 32 bytes (whole sectors).
+
+// dW rows of one chunk: out[c0 + m][n] = acc, fp32 or bf16.
 struct EpiStoreRows {
   struct Params {
     void* out;
@@ -353,26 +349,33 @@ struct EpiStoreRows {
   };
   __device__ __forceinline__ static void prefetch(const Params&, int, int, int, int) {}
   __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
-                                             int quad, int lane, float* xbuf) {
-    const int rbase = row0 + quad * 32;
+                                             int quad, int lane) {
+    const int rq = lane >> 2, cs = (lane & 3) * 2;
 #pragma unroll 1
     for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
       const int col0 = n0 + c * 32;
       if (col0 >= p.cols) break;  // warp-uniform
-      float v[32];
-      tmem_ld32(taddr + c * 32, v);
-      __syncwarp();
-      xpose_put(xbuf, lane, v);
-      __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = i * 4 + (lane >> 3), j = lane & 7;
-        const int col = col0 + 4 * j;
-        if (rbase + r < p.rows && col < p.cols) {
-          const size_t o = static_cast<size_t>(p.row_off + rbase + r) * p.ld + col;
-          const float4 val = xpose_get(xbuf, r, j);
-          if (p.out_fp32) *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = val;
-          else st_global_bf16x4(static_cast<__nv_bfloat16*>(p.out) + o, val);
+      for (int h = 0; h < 2; ++h) {
+        float v[16];
+        tmem_ld16x32(taddr + (static_cast<uint32_t>(16 * h) << 16) + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = row0 + quad * 32 + 16 * h + 8 * e + rq;
+          if (r >= p.rows) continue;
+          const size_t orow = static_cast<size_t>(p.row_off + r) * p.ld;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int col = col0 + 8 * j;
+            if (col >= p.cols) continue;
+            const float a = v[4 * j + 2 * e], b = v[4 * j + 2 * e + 1];
+            if (p.out_fp32)
+              *reinterpret_cast<float2*>(static_cast<float*>(p.out) + orow + col + cs) =
+                  make_float2(a, b);
+            else
+              *reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) + orow + col + cs) =
+                  pack_bf16x2(a, b);
+          }
         }
       }
     }
@@ -402,39 +405,43 @@ struct EpiAccumRows {
     }
   }
   __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
-                                             int quad, int lane, float* xbuf) {
-    const int rbase = row0 + quad * 32;
+                                             int quad, int lane) {
+    const int rq = lane >> 2, cs = (lane & 3) * 2;
+    const bool rd = p.mode == 2 || p.mode == 3, wr_part = p.mode == 1 || p.mode == 2;
 #pragma unroll 1
     for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
       const int col0 = n0 + c * 32;
       if (col0 >= p.cols) break;  // warp-uniform
-      float v[32];
-      tmem_ld32(taddr + c * 32, v);
-      __syncwarp();
-      xpose_put(xbuf, lane, v);
-      __syncwarp();
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = i * 4 + (lane >> 3), j = lane & 7;
-        const int col = col0 + 4 * j;
-        if (rbase + r < p.rows && col < p.cols) {
-          const size_t o = static_cast<size_t>(rbase + r) * p.ld + col;
-          float4 val = xpose_get(xbuf, r, j);
-          if (p.mode == 2 || p.mode == 3) {
-            const float4 prev = *reinterpret_cast<const float4*>(p.part + o);
-            val.x += prev.x;
-            val.y += prev.y;
-            val.z += prev.z;
-            val.w += prev.w;
+      for (int h = 0; h < 2; ++h) {
+        float v[16];
+        tmem_ld16x32(taddr + (static_cast<uint32_t>(16 * h) << 16) + c * 32, v);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = row0 + quad * 32 + 16 * h + 8 * e + rq;
+          if (r >= p.rows) continue;
+          const size_t orow = static_cast<size_t>(r) * p.ld;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int col = col0 + 8 * j;
+            if (col >= p.cols) continue;
+            float a = v[4 * j + 2 * e], b = v[4 * j + 2 * e + 1];
+            float2* pp = reinterpret_cast<float2*>(p.part + orow + col + cs);
+            if (rd) {
+              const float2 o = *pp;
+              a += o.x;
+              b += o.y;
+            }
+            if (wr_part)
+              *pp = make_float2(a, b);
+            else
+              *reinterpret_cast<uint32_t*>(p.out + orow + col + cs) = pack_bf16x2(a, b);
           }
-          if (p.mode == 1 || p.mode == 2) *reinterpret_cast<float4*>(p.part + o) = val;
-          else st_global_bf16x4(p.out + o, val);
         }
       }
     }
   }
 };
-
 
 // ====================================================================
 // Launch descriptor: up to three GEMM problems served by one persistent
@@ -456,6 +463,7 @@ constexpr int TC_SLOTS = 4;  // depth of the tile-id ring
 
 struct TcProblem {
   int kind;
+  int a_blocked, b_blocked;  // A / B use 3-D blocked tensor maps
   int m_tiles, n_tiles;   // 256 x 256 tiles
   int num_kb;             // K / 64, rounded up
   int m_fastest;          // tile order inside the problem
@@ -540,9 +548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + TC_STAGES * TC_A_BYTES;
-  float* xpose = reinterpret_cast<float*>(sB + TC_STAGES * TC_B_BYTES);  // [EPI_WARPS][32*32]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * TC_B_BYTES +
-                                               TC_EPI_WARPS * TC_XPOSE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + TC_STAGES * TC_B_BYTES);
   uint64_t* full = bars;                       // [STAGES] TMA -> MMA (even CTA's are used)
   uint64_t* empty = full + TC_STAGES;          // [STAGES] MMA -> TMA (each CTA)
   uint64_t* tfull = empty + TC_STAGES;         // [2] MMA -> epilogue (each CTA)
@@ -639,8 +645,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           }
           const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * TC_STAGE_BYTES);
-          tma_half_stage(mA, a_mn, fbar, sA + stage * TC_A_BYTES, m0, kb * TC_BK + P.a_k_off);
-          tma_half_stage(mB, b_mn, fbar, sB + stage * TC_B_BYTES, n0, kb * TC_BK + P.b_k_off);
+          tma_half_stage(mA, a_mn, P.a_blocked, fbar, sA + stage * TC_A_BYTES, m0,
+                         kb * TC_BK + P.a_k_off);
+          tma_half_stage(mB, b_mn, P.b_blocked, fbar, sB + stage * TC_B_BYTES, n0,
+                         kb * TC_BK + P.b_k_off);
           if (TC_PREFETCH_KB > 0 && kb + TC_PREFETCH_KB < P.num_kb) {
             // keep the L2 a few k-blocks ahead of the copies (HBM misses become L2 hits)
             const int kp = (kb + TC_PREFETCH_KB) * TC_BK;
@@ -732,7 +740,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     const int quad = warp & 3;         // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // which 128 accumulator columns
     const int rbase = static_cast<int>(rank) * TC_HM;
-    float* xbuf = xpose + (warp - 2) * (TC_XPOSE_BYTES / 4);
     int slot = 0, it = 0;
     uint32_t sph = 0;
     while (true) {
@@ -762,7 +769,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * TC_BN +
                              half * TC_EPI_COLS;
       dispatch_epilogue(L, P.kind, [&](auto epi, const auto& prm) {
-        decltype(epi)::run(prm, taddr, row0, n0, quad, lane, xbuf);
+        decltype(epi)::run(prm, taddr, row0, n0, quad, lane);
       });
       tc_fence_before();
       __syncwarp();
