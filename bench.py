@@ -39,7 +39,10 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from lm_head_projection_b200.workloads import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+from lm_head_projection_b200.workloads import (CE_WORKLOADS, HEADLINE, WORKLOADS,  # noqa: E402
+                                               make_inputs)
+
+ALL_WORKLOADS = {**WORKLOADS, **CE_WORKLOADS}
 
 METRIC = "fwd+bwd tokens/s at H=4096,V=128256 bf16; % of roofline (tensor/HBM)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -92,7 +95,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
+    ap.add_argument("--workload", default=HEADLINE, choices=list(ALL_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=8)
@@ -185,6 +188,12 @@ def oracle_sample(w, rows, seed=123):
 
     inp = make_inputs(w.with_(BT=rows, seed=seed), device="cpu")
     f = lambda t: None if t is None else t.float().numpy().astype(np.float64)
+    if w.ce:
+        args = (f(inp["X"]), f(inp["W"]), f(inp["b"]), inp["target"].numpy())
+        kw = dict(ignore_index=inp["ignore_index"], temperature=inp["temperature"],
+                  reduction=inp["reduction"], compute_dW=inp["compute_dW"],
+                  compute_db=inp["compute_db"], ce=True)
+        return args, kw
     args = (f(inp["X"]), f(inp["W"]), f(inp["b"]), f(inp["Q"]))
     kw = dict(shift_labels=None if inp["shift_labels"] is None else inp["shift_labels"].numpy(),
               ignore_index=inp["ignore_index"], temperature=inp["temperature"], eps=inp["eps"],
@@ -205,10 +214,12 @@ def host_threads():
 
 
 def time_oracle(args, kw):
-    from oracle import forward_backward as oracle_fb
+    from oracle import ce_forward_backward, forward_backward
 
+    kw = dict(kw)
+    fn = ce_forward_backward if kw.pop("ce", False) else forward_backward
     t0 = time.perf_counter()
-    oracle_fb(*args, **kw)
+    fn(*args, **kw)
     return time.perf_counter() - t0
 
 
@@ -226,15 +237,27 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=dev)
-    w = WORKLOADS[args.workload].with_(seed=WORKLOADS[args.workload].seed + rank)
+    w = ALL_WORKLOADS[args.workload].with_(seed=ALL_WORKLOADS[args.workload].seed + rank)
     inp = make_inputs(w, device=dev)
     X, W, b, Q, lab = inp["X"], inp["W"], inp["b"], inp["Q"], inp["shift_labels"]
+    tgt = inp.get("target")
     dt_code = pkg.DTYPES[X.dtype]
     compute_db = inp["compute_db"]
-    r0 = pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
-                              inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
-                              compute_db=compute_db, accum_fp32=inp["accum_fp32"],
-                              check_status=True)
+
+    def api_call(out=None, workspace=None, check_status=False):
+        """The public Python API call a user makes for this workload."""
+        if w.ce:
+            return pkg.cross_entropy_forward_backward(
+                X, W, b, tgt, inp["ignore_index"], inp["temperature"], inp["reduction"],
+                compute_dW=inp["compute_dW"], compute_db=compute_db,
+                accum_fp32=inp["accum_fp32"], out=out, workspace=workspace,
+                check_status=check_status)
+        return pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
+                                    inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
+                                    compute_db=compute_db, accum_fp32=inp["accum_fp32"],
+                                    out=out, workspace=workspace, check_status=check_status)
+
+    r0 = api_call(check_status=True)
     ws = r0["workspace"]
     out = {k: r0[k] for k in ("loss", "dX", "dW", "db")}
     stream = torch.cuda.current_stream(dev)
@@ -243,9 +266,14 @@ def run_ours(args):
                  inp["temperature"], inp["eps"], pkg.REDUCTIONS[inp["reduction"]],
                  inp["compute_dW"], compute_db, inp["accum_fp32"], p(out["loss"]), p(out["dX"]),
                  p(out["dW"]), p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
+    ce_args = (p(X), p(W), p(b), p(tgt), inp["ignore_index"], w.BT, w.H, w.V, dt_code,
+               inp["temperature"], pkg.REDUCTIONS[inp["reduction"]], inp["compute_dW"],
+               compute_db, inp["accum_fp32"], p(out["loss"]), p(out["dX"]), p(out["dW"]),
+               p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
 
     def step():
-        s = pkg.flkl_forward_backward(*call_args)
+        s = (pkg.flkl_ce_forward_backward(*ce_args) if w.ce
+             else pkg.flkl_forward_backward(*call_args))
         if s != 0:
             raise pkg.FlklError(s, "flkl_forward_backward")
 
@@ -285,7 +313,8 @@ def run_ours(args):
     per_kind = {}  # kind -> [ms, launches, gemm flops]
     launches_per_step = 0
     for _ in range(args.steps):
-        st, kinds, flops, n = pkg.flkl_forward_backward_profiled(*call_args, events, cap)
+        st, kinds, flops, n = pkg.flkl_forward_backward_profiled(*call_args, events, cap,
+                                                                 ce_target=p(tgt))
         if st != 0:
             raise pkg.FlklError(st, "flkl_forward_backward_profiled")
         launches_per_step = n
@@ -337,33 +366,27 @@ def run_ours(args):
                      "peaks": peaks_src}
 
     # ---------------- end to end: batch from pinned host memory, loss back
-    hX = X.cpu().pin_memory()
-    hQ = Q.cpu().pin_memory()
-    hL = None if lab is None else lab.cpu().pin_memory()
+    # the step's batch: X, and the teacher Q (or the targets) and the labels
+    batch = [t for t in (X, Q, lab, tgt) if t is not None]
+    hosts = [t.cpu().pin_memory() for t in batch]
     hloss = torch.empty((), dtype=torch.float32).pin_memory()
-    h2d = hX.numel() * hX.element_size() + hQ.numel() * hQ.element_size() + \
-        (0 if hL is None else hL.numel() * 8)
+    h2d = sum(h.numel() * h.element_size() for h in hosts)
+
+    def copy_batch():
+        for d, h in zip(batch, hosts):
+            d.copy_(h, non_blocking=True)
+
     for _ in range(max(1, args.warmup)):
-        X.copy_(hX, non_blocking=True)
-        Q.copy_(hQ, non_blocking=True)
-        pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
-                             inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
-                             compute_db=compute_db, accum_fp32=inp["accum_fp32"], out=out,
-                             workspace=ws)
+        copy_batch()
+        api_call(out=out, workspace=ws)
         hloss.copy_(out["loss"], non_blocking=True)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(args.steps):
-        X.copy_(hX, non_blocking=True)
-        Q.copy_(hQ, non_blocking=True)
-        if hL is not None:
-            lab.copy_(hL, non_blocking=True)
-        pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
-                             inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
-                             compute_db=compute_db, accum_fp32=inp["accum_fp32"], out=out,
-                             workspace=ws)
+        copy_batch()
+        api_call(out=out, workspace=ws)
         hloss.copy_(out["loss"], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -406,7 +429,7 @@ def algorithmic_bytes(w) -> float:
     """X, W, Q and labels read once, dX and dW/db written once."""
     e = 4 if w.dtype == "fp32" else 2
     pe = 4 if (w.accum_fp32 or w.dtype == "fp32") else 2
-    b = w.BT * w.H * e * 2 + w.V * w.H * e + w.BT * w.V * e
+    b = w.BT * w.H * e * 2 + w.V * w.H * e + (w.BT * 8 if w.ce else w.BT * w.V * e)
     if w.compute_dW:
         b += w.V * w.H * pe
     if w.bias:
@@ -423,7 +446,7 @@ def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    w = WORKLOADS[args.workload]
+    w = ALL_WORKLOADS[args.workload]
     rows = max(1, min(args.ref_rows, w.BT))
     oa, okw = oracle_sample(w, rows)
     for _ in range(args.warmup):

@@ -124,6 +124,30 @@ FLKL_API flkl_status flkl_forward_backward(const void* X, const void* W, const v
                                   float* loss, void* dX, void* dW, void* db, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* Fused linear-head + cross-entropy loss: flkl_forward_backward with a
+ * one-hot teacher at target[r], i.e. KL(onehot || P) = -log p_{r, target[r]}
+ * (the cross-entropy of fused_linear_cross_entropy, which the
+ * FusedLinearKLDivLoss page names in its Summary as the source of its chunk
+ * geometry).  No teacher tensor is read.
+ *
+ *  target  device, [BT] int64: the class of each row; a row whose target
+ *          equals ignore_index is dropped (it is the row mask too).  A
+ *          target outside [0, V) that is not ignore_index gives its row no
+ *          teacher mass: the row's loss and dX are 0 (such targets are not
+ *          validated).
+ *  Other arguments, outputs, workspace (flkl_workspace_size with the same
+ *  sizes), reductions (batchmean divides by the kept rows, which is torch's
+ *  cross_entropy "mean"), temperature and errors: as flkl_forward_backward;
+ *  eps does not apply.  Loss = sum over kept rows of
+ *  (logsumexp(z_r/T) - z_{r,target}/T) / D, dz = (p - onehot) / (T D). */
+FLKL_API flkl_status flkl_ce_forward_backward(const void* X, const void* W, const void* b,
+                                              const int64_t* target, int64_t ignore_index,
+                                              int64_t BT, int64_t H, int64_t V, int dtype,
+                                              float temperature, int reduction, int compute_dW,
+                                              int compute_db, int accum_fp32, float* loss,
+                                              void* dX, void* dW, void* db, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
 /* Kinds of launches reported by flkl_forward_backward_profiled. */
 typedef enum {
   FLKL_LAUNCH_PREPARE = 0,  /* valid-row count and divisor                   */
@@ -148,13 +172,16 @@ typedef enum {
  * the number of launches of the call (which may exceed capacity; the extra
  * ones are not recorded).  Same results and errors as
  * flkl_forward_backward, plus FLKL_ERR_INVALID_ARG for a null
- * events/kinds/flops/n_launches or a negative capacity. */
+ * events/kinds/flops/n_launches or a negative capacity.  With ce_target
+ * non-NULL (and Q and shift_labels NULL) it profiles flkl_ce_forward_backward
+ * instead (eps ignored). */
 FLKL_API flkl_status flkl_forward_backward_profiled(
     const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
     int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
     float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
     void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
-    void** events, int* kinds, double* flops, int capacity, int* n_launches);
+    void** events, int* kinds, double* flops, int capacity, int* n_launches,
+    const int64_t* ce_target);
 
 /* Size of the fixed device scratch used by flkl_forward_backward_noalloc. */
 #define FLKL_NOALLOC_SCRATCH_BYTES (128u << 20)

@@ -20,6 +20,7 @@ __all__ = [
     "flkl_forward_backward_profiled", "LAUNCH_KINDS", "flkl_forward_backward_noalloc",
     "flkl_device_status", "flkl_set_wait_limit_ms", "flkl_wait_selftest", "flkl_status_string",
     "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
+    "flkl_ce_forward_backward", "cross_entropy_forward_backward", "FusedLinearCrossEntropyLoss",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -66,7 +67,16 @@ def _lib():
             c.c_void_p, c.c_size_t, c.c_void_p]                  # ws bytes stream
         lib.flkl_forward_backward_profiled.restype = c.c_int
         lib.flkl_forward_backward_profiled.argtypes = list(lib.flkl_forward_backward.argtypes) + [
-            c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_void_p]
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_void_p, c.c_void_p]
+        lib.flkl_ce_forward_backward.restype = c.c_int
+        lib.flkl_ce_forward_backward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p,                  # X W b
+            c.c_void_p, c.c_int64,                               # target ignore_index
+            c.c_int64, c.c_int64, c.c_int64, c.c_int,            # BT H V dtype
+            c.c_float, c.c_int,                                  # T reduction
+            c.c_int, c.c_int, c.c_int,                           # dW db accum_fp32
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,      # loss dX dW db
+            c.c_void_p, c.c_size_t, c.c_void_p]                  # ws bytes stream
         lib.flkl_forward_backward_noalloc.restype = c.c_int
         lib.flkl_forward_backward_noalloc.argtypes = (
             list(lib.flkl_forward_backward.argtypes[:20]) + [c.c_void_p])
@@ -108,6 +118,17 @@ def flkl_forward_backward(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtyp
         int(workspace_bytes), stream)
 
 
+def flkl_ce_forward_backward(X, W, b, target, ignore_index, BT, H, V, dtype, temperature,
+                             reduction, compute_dW, compute_db, accum_fp32, loss, dX, dW, db,
+                             workspace, workspace_bytes, stream) -> int:
+    """The cross-entropy C entry point (one-hot teacher at target[r]) with raw
+    integer pointers; returns the status."""
+    return _lib().flkl_ce_forward_backward(
+        X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), int(reduction), int(bool(compute_dW)), int(bool(compute_db)),
+        int(bool(accum_fp32)), loss, dX, dW, db, workspace, int(workspace_bytes), stream)
+
+
 def flkl_forward_backward_noalloc(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
                                   temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
                                   loss, dX, dW, db, stream) -> int:
@@ -127,7 +148,7 @@ LAUNCH_KINDS = ("prepare", "stats", "combine", "loss", "grad", "dW", "dX", "db",
 def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
                                    temperature, eps, reduction, compute_dW, compute_db,
                                    accum_fp32, loss, dX, dW, db, workspace, workspace_bytes,
-                                   stream, events, capacity):
+                                   stream, events, capacity, ce_target=None):
     """The profiled C entry point.  ``events`` is a list of 2*capacity
     torch.cuda.Event(enable_timing=True), each recorded once beforehand (torch
     creates the CUDA event lazily).  Returns (status, kinds, flops, n) with the
@@ -141,7 +162,7 @@ def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H
         X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
         float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
         int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
-        int(workspace_bytes), stream, ev, kinds, flops, int(capacity), c.byref(n))
+        int(workspace_bytes), stream, ev, kinds, flops, int(capacity), c.byref(n), ce_target)
     k = min(n.value, capacity)
     return st, [kinds[i] for i in range(k)], [flops[i] for i in range(k)], n.value
 
@@ -297,3 +318,111 @@ class FusedLinearKLDivLoss(torch.nn.Module):
         return _FusedLinearKLDivFunction.apply(_input, lin_weight, bias, target_probs,
                                                shift_labels, self.ignore_index, self.temperature,
                                                self.eps, self.reduction, self.accum_fp32)
+
+
+def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor],
+                                   target: torch.Tensor, ignore_index: int = -100,
+                                   temperature: float = 1.0, reduction: str = "batchmean",
+                                   compute_dW: bool = True, compute_db: bool = False,
+                                   accum_fp32: bool = True, out: Optional[dict] = None,
+                                   workspace: Optional[torch.Tensor] = None,
+                                   stream: Optional[torch.cuda.Stream] = None,
+                                   check_status: bool = False) -> dict:
+    """Fused linear + cross-entropy (one-hot teacher at ``target``) in one call.
+    ``reduction="batchmean"`` divides by the kept rows (torch's cross_entropy
+    "mean").  Same outputs and conventions as :func:`forward_backward`."""
+    if reduction not in REDUCTIONS:
+        raise ValueError(f"unknown reduction {reduction!r}")
+    if X.dtype not in DTYPES:
+        raise ValueError(f"dtype {X.dtype} not supported (float32 or bfloat16)")
+    dev = X.device
+    BT, H = X.shape
+    V = W.shape[0]
+    dt = X.dtype
+    _check_dev("X", X, dt, (BT, H), dev)
+    _check_dev("W", W, dt, (V, H), dev)
+    _check_dev("target", target, torch.int64, (BT,), dev)
+    if b is not None:
+        _check_dev("b", b, dt, (V,), dev)
+    compute_db = bool(compute_db and b is not None)
+    pdt = torch.float32 if (accum_fp32 or dt == torch.float32) else dt
+    out = {} if out is None else out
+    loss = out.get("loss")
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=dev)
+    dX = out.get("dX")
+    if dX is None:
+        dX = torch.empty_like(X)
+    dW = out.get("dW") if compute_dW else None
+    if compute_dW and dW is None:
+        dW = torch.empty((V, H), dtype=pdt, device=dev)
+    db = out.get("db") if compute_db else None
+    if compute_db and db is None:
+        db = torch.empty((V,), dtype=pdt, device=dev)
+    need = flkl_workspace_size(BT, H, V, DTYPES[dt], compute_dW, compute_db)
+    if need == 0:
+        raise FlklError(1, "flkl_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    status = flkl_ce_forward_backward(
+        _ptr(X), _ptr(W), _ptr(b), _ptr(target), ignore_index, BT, H, V, DTYPES[dt],
+        temperature, REDUCTIONS[reduction], compute_dW, compute_db, accum_fp32, _ptr(loss),
+        _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace), workspace.numel(), st.cuda_stream)
+    if status != FLKL_OK:
+        raise FlklError(status, "flkl_ce_forward_backward")
+    if check_status:
+        s = flkl_device_status(_ptr(workspace), st.cuda_stream)
+        if s != FLKL_OK:
+            raise FlklError(s, "flkl_ce_forward_backward (device)")
+    return {"loss": loss, "dX": dX, "dW": dW, "db": db, "workspace": workspace}
+
+
+class _FusedLinearCEFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, X, W, b, target, ignore_index, temperature, reduction, accum_fp32):
+        r = cross_entropy_forward_backward(
+            X.contiguous(), W.contiguous(), None if b is None else b.contiguous(),
+            target.contiguous(), ignore_index, temperature, reduction,
+            compute_dW=ctx.needs_input_grad[1],
+            compute_db=b is not None and ctx.needs_input_grad[2], accum_fp32=accum_fp32)
+        ctx.save_for_backward(r["dX"], r["dW"], r["db"])
+        ctx.w_dtype = W.dtype
+        return r["loss"]
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        dX, dW, db = ctx.saved_tensors
+        if not bool((grad_out == 1).all()):
+            dX = dX * grad_out.to(dX.dtype)
+            dW = None if dW is None else dW * grad_out.to(dW.dtype)
+            db = None if db is None else db * grad_out.to(db.dtype)
+        if dW is not None:
+            dW = dW.to(ctx.w_dtype)
+        if db is not None:
+            db = db.to(ctx.w_dtype)
+        return dX, dW, db, None, None, None, None, None
+
+
+class FusedLinearCrossEntropyLoss(torch.nn.Module):
+    """Fused vocabulary-head projection + cross-entropy with gradient in
+    forward (the one-hot-teacher case of FusedLinearKLDivLoss).
+
+    ``forward(lin_weight, _input, target, bias=None)``; rows whose target
+    equals ``ignore_index`` are dropped; ``reduction`` "batchmean" (kept-row
+    mean, torch's "mean"), "mean" (per element) or "sum".
+    """
+
+    def __init__(self, ignore_index: int = -100, reduction: str = "batchmean",
+                 temperature: float = 1.0, accum_dtype: Optional[torch.dtype] = None):
+        super().__init__()
+        if reduction not in ("batchmean", "mean", "sum"):
+            raise ValueError(f"reduction {reduction!r} is not supported")
+        self.ignore_index = ignore_index
+        self.reduction = reduction
+        self.temperature = temperature
+        self.accum_fp32 = accum_dtype == torch.float32
+
+    def forward(self, lin_weight, _input, target, bias=None):
+        return _FusedLinearCEFunction.apply(_input, lin_weight, bias, target, self.ignore_index,
+                                            self.temperature, self.reduction, self.accum_fp32)

@@ -266,7 +266,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
                    long long ignore_index, int BT, int H, int V, float T, float eps,
                    int compute_dW, int compute_db, int accum_fp32, float* loss,
                    __nv_bfloat16* dX, void* dW, void* db, uint8_t* ws, cudaStream_t st,
-                   Recorder* rec) {
+                   Recorder* rec, const int64_t* target) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   int* counters = reinterpret_cast<int*>(ws + P.off_cnt);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
@@ -294,7 +294,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     L.err_flag = &ctl->err;
     L.wait_limit_ns = g_wait_limit_ns;
     L.stats = EpiStats::Params{Q, b, BT, V, t_scale, eps, stats,
-                               static_cast<long long>(P.n_stat) * BT};
+                               static_cast<long long>(P.n_stat) * BT, target};
     return L;
   };
   auto chunk_c0 = [&](long long c) { return static_cast<int>(c * P.Vc); };
@@ -304,8 +304,8 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
   // pass-2 problem of chunk c: logits of the chunk again -> G staging
   auto add_grad = [&](TcLaunch& L, TcMaps& maps, long long c) {
     const int c0 = chunk_c0(c);
-    L.grad = EpiGrad::Params{Q,     b,     BT,   V,     c0,     ldg,   Gbuf[c & 1],
-                             t_scale, lse2, coefS, coefQ, dbpart};
+    L.grad = EpiGrad::Params{Q,     b,     BT,    V,     c0,     ldg,   Gbuf[c & 1],
+                             t_scale, lse2, coefS, coefQ, dbpart, target};
     return add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, c0, 0);
   };
 
@@ -373,7 +373,8 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
 flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* b, const float* Q,
                     const int64_t* labels, long long ignore_index, int BT, int H, int V, float T,
                     float eps, int compute_dW, int compute_db, float* loss, float* dX, float* dW,
-                    float* db, uint8_t* ws, cudaStream_t st, Recorder* rec) {
+                    float* db, uint8_t* ws, cudaStream_t st, Recorder* rec,
+                    const int64_t* target) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
   float* rows = reinterpret_cast<float*>(ws + P.off_rows);
@@ -390,7 +391,7 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
   {
   Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
   k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
-      X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT);
+      X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT, target);
   FLKL_CUDA(cudaGetLastError());
   }
   {
@@ -413,7 +414,7 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
     {
     Rec r_(rec, 4, 2.0 * BT * static_cast<double>(Vw) * H);
     k_simt_grad<<<dim3(static_cast<unsigned>(cdiv(Vw, ST_T)), mt), 256, 0, st>>>(
-        X, W, b, Q, BT, H, V, c0, Vw, t_scale, lse2, coefS, coefQ, G, ldg, dbpart);
+        X, W, b, Q, BT, H, V, c0, Vw, t_scale, lse2, coefS, coefQ, G, ldg, dbpart, target);
     FLKL_CUDA(cudaGetLastError());
     }
     if (compute_dW) {
@@ -500,7 +501,14 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
                                   int64_t H, int64_t V, int dtype, float temperature, float eps,
                                   int reduction, int compute_dW, int compute_db, int accum_fp32,
                                   float* loss, void* dX, void* dW, void* db, void* workspace,
-                                  size_t workspace_bytes, void* stream, Recorder* rec) {
+                                  size_t workspace_bytes, void* stream, Recorder* rec,
+                                  const int64_t* target = nullptr) {
+  // Cross-entropy mode (target set): the teacher is one-hot at target[row],
+  // Q is not read and the target doubles as the row mask.
+  if (target != nullptr) {
+    if (Q != nullptr || shift_labels != nullptr) return FLKL_ERR_INVALID_ARG;
+    shift_labels = target;
+  }
   // ---- scalar arguments
   if (dtype != FLKL_DTYPE_F32 && dtype != FLKL_DTYPE_BF16) return FLKL_ERR_INVALID_ARG;
   if (reduction == FLKL_REDUCTION_NONE) return FLKL_ERR_UNSUPPORTED;
@@ -515,7 +523,8 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
   if (H % vec != 0 || V % vec != 0) return FLKL_ERR_UNSUPPORTED;
   // ---- pointers
   if (W == nullptr || loss == nullptr) return FLKL_ERR_INVALID_ARG;
-  if (BT > 0 && (X == nullptr || Q == nullptr || dX == nullptr)) return FLKL_ERR_INVALID_ARG;
+  if (BT > 0 && (X == nullptr || (Q == nullptr && target == nullptr) || dX == nullptr))
+    return FLKL_ERR_INVALID_ARG;
   if ((compute_dW != 0) != (dW != nullptr)) return FLKL_ERR_INVALID_ARG;
   if ((compute_db != 0) != (db != nullptr)) return FLKL_ERR_INVALID_ARG;
   if (compute_db && b == nullptr) return FLKL_ERR_INVALID_ARG;
@@ -565,13 +574,13 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
     return run_tc(P, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
                   static_cast<const __nv_bfloat16*>(b), static_cast<const __nv_bfloat16*>(Q),
                   shift_labels, ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db,
-                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st, rec);
+                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st, rec, target);
   }
   return run_f32(P, static_cast<const float*>(X), static_cast<const float*>(W),
                  static_cast<const float*>(b), static_cast<const float*>(Q), shift_labels,
                  ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db, loss,
                  static_cast<float*>(dX), static_cast<float*>(dW), static_cast<float*>(db), ws,
-                 st, rec);
+                 st, rec, target);
 }
 
 // Fixed scratch of flkl_forward_backward_noalloc (see flkl.h): part of the
@@ -639,20 +648,37 @@ flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, c
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr);
 }
 
+flkl_status flkl_ce_forward_backward(const void* X, const void* W, const void* b,
+                                     const int64_t* target, int64_t ignore_index, int64_t BT,
+                                     int64_t H, int64_t V, int dtype, float temperature,
+                                     int reduction, int compute_dW, int compute_db, int accum_fp32,
+                                     float* loss, void* dX, void* dW, void* db, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (BT > 0 && target == nullptr) return FLKL_ERR_INVALID_ARG;
+  return forward_backward_impl(X, W, b, nullptr, nullptr, ignore_index, BT, H, V, dtype,
+                               temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
+                               BT > 0 ? target : nullptr);
+}
+
 flkl_status flkl_forward_backward_profiled(
     const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
     int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
     float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
     void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
-    void** events, int* kinds, double* flops, int capacity, int* n_launches) {
+    void** events, int* kinds, double* flops, int capacity, int* n_launches,
+    const int64_t* ce_target) {
   if (events == nullptr || kinds == nullptr || flops == nullptr || n_launches == nullptr ||
       capacity < 0)
     return FLKL_ERR_INVALID_ARG;
   Recorder r{reinterpret_cast<cudaEvent_t*>(events), kinds, flops, capacity, 0,
              static_cast<cudaStream_t>(stream)};
+  if (ce_target != nullptr && BT == 0) ce_target = nullptr;
+  if (ce_target == nullptr && Q == nullptr && BT > 0) return FLKL_ERR_INVALID_ARG;
   const flkl_status s = forward_backward_impl(
       X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype, temperature, eps, reduction,
-      compute_dW, compute_db, accum_fp32, loss, dX, dW, db, workspace, workspace_bytes, stream, &r);
+      compute_dW, compute_db, accum_fp32, loss, dX, dW, db, workspace, workspace_bytes, stream, &r,
+      ce_target);
   *n_launches = r.count;
   return s;
 }

@@ -51,13 +51,15 @@ __device__ __forceinline__ void simt_tile_mma(const float* __restrict__ A, long 
 }
 
 // Pass 1 (fp32): z tile = X W^T + b over 64 vocabulary columns; per-row
-// statistics of the tile in the same form as the tensor-core path.
+// statistics of the tile in the same form as the tensor-core path.  With
+// `target` set, the teacher is one-hot at target[row] (Q unused).
 __global__ void __launch_bounds__(256) k_simt_stats(const float* __restrict__ X,
                                                     const float* __restrict__ W,
                                                     const float* __restrict__ bias,
                                                     const float* __restrict__ Q, int BT, int H,
                                                     int V, float t_scale, float eps,
-                                                    float* __restrict__ st, long long plane) {
+                                                    float* __restrict__ st, long long plane,
+                                                    const int64_t* __restrict__ target) {
   __shared__ float Zs[ST_T][ST_T + 1];
   const int mb = blockIdx.y, nb = blockIdx.x;
   const int m0 = mb * ST_T, n0 = nb * ST_T;
@@ -81,7 +83,8 @@ __global__ void __launch_bounds__(256) k_simt_stats(const float* __restrict__ X,
       float s = 0.f;
       for (int c = 0; c < ST_T && n0 + c < V; ++c) {
         const float z = Zs[r][c] + (bias ? bias[n0 + c] : 0.f);
-        const float q = Q[static_cast<size_t>(row) * V + n0 + c];
+        const float q = target != nullptr ? (target[row] == n0 + c ? 1.f : 0.f)
+                                          : Q[static_cast<size_t>(row) * V + n0 + c];
         s += exp2f(z * t_scale - m);
         A = fmaf(q, z, A);
         S += q;
@@ -109,7 +112,8 @@ __global__ void __launch_bounds__(256) k_simt_grad(const float* __restrict__ X,
                                                    const float* __restrict__ coefS,
                                                    const float* __restrict__ coefQ,
                                                    float* __restrict__ G, int ldg,
-                                                   float* __restrict__ dbpart) {
+                                                   float* __restrict__ dbpart,
+                                                   const int64_t* __restrict__ target) {
   __shared__ float Gs[ST_T][ST_T + 1];
   const int mb = blockIdx.y, nb = blockIdx.x;
   const int m0 = mb * ST_T, n0 = nb * ST_T;  // n0 chunk-relative
@@ -125,7 +129,9 @@ __global__ void __launch_bounds__(256) k_simt_grad(const float* __restrict__ X,
       float g = 0.f;
       if (row < BT && col < Vw) {
         const float t = (acc[i][j] + (bias ? bias[gcol] : 0.f)) * t_scale;
-        g = coefS[row] * exp2f(t - lse2[row]) - coefQ[row] * Q[static_cast<size_t>(row) * V + gcol];
+        const float q = target != nullptr ? (target[row] == gcol ? 1.f : 0.f)
+                                          : Q[static_cast<size_t>(row) * V + gcol];
+        g = coefS[row] * exp2f(t - lse2[row]) - coefQ[row] * q;
         G[static_cast<size_t>(row) * ldg + col] = g;
       }
       Gs[r][c] = g;

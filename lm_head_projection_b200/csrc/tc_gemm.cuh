@@ -165,18 +165,19 @@ __device__ __forceinline__ void load_bias32(const __nv_bfloat16* bias, int col0,
 //   A = sum q z, B2 = sum q log2 max(q, eps), S = sum q
 struct EpiStats {
   struct Params {
-    const __nv_bfloat16* Q;
+    const __nv_bfloat16* Q;     // teacher [BT][V]; null in cross-entropy mode
     const __nv_bfloat16* bias;  // may be null
     int BT, V;
     float t_scale;  // log2(e) / T
     float eps;
     float* st;      // [5][n_groups][BT], n_groups = ceil(V/128)
     long long st_plane;  // n_groups * BT
+    const int64_t* target;  // cross-entropy mode: q = one-hot at target[row]; else null
   };
   __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
                                                   int lane) {
     const int row = row0 + quad * 32 + lane;
-    if (row < p.BT && n0 < p.V) {
+    if (p.Q != nullptr && row < p.BT && n0 < p.V) {
       const __nv_bfloat16* q = p.Q + static_cast<size_t>(row) * p.V + n0;
       prefetch_l2(q);
       if (n0 + 64 < p.V) prefetch_l2(q + 64);
@@ -187,19 +188,27 @@ struct EpiStats {
     const int row = row0 + quad * 32 + lane;
     const bool rv = row < p.BT;
     if (n0 >= p.V) return;  // warp-uniform: this half of the tile is past V
-    const __nv_bfloat16* qrow = p.Q + static_cast<size_t>(rv ? row : 0) * p.V;
+    const bool ce = p.Q == nullptr;  // warp-uniform
+    const __nv_bfloat16* qrow = ce ? nullptr : p.Q + static_cast<size_t>(rv ? row : 0) * p.V;
+    long long y = (ce && rv) ? p.target[row] : -1;
+    if (y >= p.V) y = -1;  // a target outside [0, V) matches no column
     const float qmin = fmaxf(p.eps, 1.17549435e-38f);
     float m = -INFINITY, s = 0.f, A = 0.f, B2 = 0.f, S = 0.f;
     uint4 qa[4], qb[4];
-    load_chunk32(qrow, rv, n0, p.V, qa);
+    if (!ce) load_chunk32(qrow, rv, n0, p.V, qa);
 #pragma unroll 1
     for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
       const int col0 = n0 + c * 32;
       if (col0 >= p.V) break;  // warp-uniform
-      if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, col0 + 32, p.V, qb);
       float q[32], bv[32], z[32];
+      if (!ce) {
+        if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, col0 + 32, p.V, qb);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+        for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) q[i] = (col0 + i == y) ? 1.f : 0.f;
+      }
       load_bias32(p.bias, col0, p.V, bv);
       tmem_ld32(taddr + c * 32, z);
       float cm = -INFINITY;
@@ -266,12 +275,13 @@ struct EpiGrad {
     const float* coefS;  // [BT] S_r / (T D), 0 on dropped rows
     const float* coefQ;  // [BT] 1 / (T D), 0 on dropped rows
     float* dbpart;       // [row groups of 32][V] or null
+    const int64_t* target;  // cross-entropy mode (Q null): one-hot teacher at target[row]
   };
   __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
                                                   int lane) {
     const int row = row0 + quad * 32 + lane;
     const int gc = p.c0 + n0;
-    if (row < p.BT && gc < p.V) {
+    if (p.Q != nullptr && row < p.BT && gc < p.V) {
       const __nv_bfloat16* q = p.Q + static_cast<size_t>(row) * p.V + gc;
       prefetch_l2(q);
       if (gc + 64 < p.V) prefetch_l2(q + 64);
@@ -282,21 +292,29 @@ struct EpiGrad {
     const int row = row0 + quad * 32 + lane;
     const bool rv = row < p.BT;  // n0 is chunk-relative
     if (p.c0 + n0 >= p.V) return;  // warp-uniform
-    const __nv_bfloat16* qrow = p.Q + static_cast<size_t>(rv ? row : 0) * p.V;
+    const bool ce = p.Q == nullptr;  // warp-uniform
+    const __nv_bfloat16* qrow = ce ? nullptr : p.Q + static_cast<size_t>(rv ? row : 0) * p.V;
+    long long y = (ce && rv) ? p.target[row] : -1;
+    if (y >= p.V) y = -1;  // a target outside [0, V) matches no column
     const float lse2 = rv ? p.lse2[row] : 0.f;
     const float cS = rv ? p.coefS[row] : 0.f;
     const float cQ = rv ? p.coefQ[row] : 0.f;
     uint4 qa[4], qb[4];
-    load_chunk32(qrow, rv, p.c0 + n0, p.V, qa);
+    if (!ce) load_chunk32(qrow, rv, p.c0 + n0, p.V, qa);
 #pragma unroll 1
     for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
       const int col0 = n0 + c * 32;
       const int gcol0 = p.c0 + col0;
       if (gcol0 >= p.V) break;  // warp-uniform
-      if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, gcol0 + 32, p.V, qb);
       float q[32], bv[32], z[32];
+      if (!ce) {
+        if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, gcol0 + 32, p.V, qb);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+        for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) q[i] = (gcol0 + i == y) ? 1.f : 0.f;
+      }
       load_bias32(p.bias, gcol0, p.V, bv);
       tmem_ld32(taddr + c * 32, z);
 #pragma unroll

@@ -62,6 +62,7 @@ class Workload:
     ignore_frac: float = 0.0
     zero_frac: float = 0.0
     seed: int = 0
+    ce: bool = False  # cross-entropy: one-hot teacher at an integer target per row
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -111,6 +112,22 @@ WORKLOAD_ORDER = list(WORKLOADS)
 HEADLINE = "bf16_bt1024_h4096_v128256"
 
 
+# Cross-entropy workloads (the one-hot-teacher case): the headline head shape
+# with uniform targets, 10 % of rows dropped, and a small fp32 case.
+CE_WORKLOADS = {
+    "ce_bf16_bt1024_h4096_v128256": Workload(
+        "ce_bf16_bt1024_h4096_v128256", "bf16", 1024, 4096, 128256, False,
+        x_std=1.0, w_std=0.02, b_std=0.0, q_std=0.0,
+        temperature=1.0, eps=0.0, reduction="batchmean",
+        compute_dW=True, compute_db=False, accum_fp32=True, ignore_frac=0.1, ce=True),
+    "ce_fp32_bt64_h256_v1024": Workload(
+        "ce_fp32_bt64_h256_v1024", "fp32", 64, 256, 1024, True,
+        x_std=1.0, w_std=1.0 / math.sqrt(256), b_std=0.02, q_std=0.0,
+        temperature=1.0, eps=0.0, reduction="batchmean",
+        compute_dW=True, compute_db=True, accum_fp32=True, ignore_frac=0.1, ce=True),
+}
+
+
 def _gen(device, seed: int, stream: int, block: int = 0) -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(((seed * 1_000_003 + stream) * 1_000_033 + block) & 0x7FFF_FFFF_FFFF_FFFF)
@@ -135,6 +152,18 @@ def make_inputs(w: Workload, device="cpu", q_block_rows: int = 256) -> dict:
     X = _randn((w.BT, w.H), w.x_std, device, _gen(device, w.seed, _S_X), dt)
     W = _randn((w.V, w.H), w.w_std, device, _gen(device, w.seed, _S_W), dt)
     b = _randn((w.V,), w.b_std, device, _gen(device, w.seed, _S_B), dt) if w.bias else None
+
+    if w.ce:
+        target = torch.randint(0, w.V, (w.BT,), generator=_gen(device, w.seed, _S_LABELS),
+                               device=device, dtype=torch.int64)
+        n_ign = int(round(w.ignore_frac * w.BT))
+        if n_ign:
+            perm = torch.randperm(w.BT, generator=_gen(device, w.seed, _S_IGNORE), device=device)
+            target[perm[:n_ign]] = IGNORE_INDEX
+        return dict(X=X, W=W, b=b, Q=None, target=target, shift_labels=None,
+                    ignore_index=IGNORE_INDEX, temperature=w.temperature, eps=w.eps,
+                    reduction=w.reduction, compute_dW=w.compute_dW,
+                    compute_db=w.compute_db and w.bias, accum_fp32=w.accum_fp32)
 
     soft_dtype = torch.float64 if w.dtype == "fp32" else torch.float32
     Q = torch.empty((w.BT, w.V), dtype=dt, device=device)
@@ -173,12 +202,12 @@ def make_inputs(w: Workload, device="cpu", q_block_rows: int = 256) -> dict:
 def small_case(dtype="bf16", BT=133, H=192, V=1000, bias=True, reduction="batchmean",
                temperature=1.0, eps=1e-10, ignore_frac=0.0, zero_frac=0.0,
                compute_dW=True, compute_db=None, q_std=2.0, x_std=1.0, w_std=None,
-               b_std=0.02, seed=0) -> Workload:
+               b_std=0.02, seed=0, ce=False) -> Workload:
     """A small workload for parity tests: several tiles and a ragged tail."""
     if w_std is None:
         w_std = 1.0 / math.sqrt(H)
     if compute_db is None:
         compute_db = bias
-    return Workload(f"small_{dtype}_{BT}x{H}x{V}", dtype, BT, H, V, bias, x_std, w_std,
-                    b_std, q_std, temperature, eps, reduction, compute_dW, compute_db,
-                    True, ignore_frac, zero_frac, seed)
+    return Workload(f"small_{'ce_' if ce else ''}{dtype}_{BT}x{H}x{V}", dtype, BT, H, V, bias,
+                    x_std, w_std, b_std, q_std, temperature, eps, reduction, compute_dW,
+                    compute_db, True, ignore_frac, zero_frac, seed, ce)

@@ -217,3 +217,70 @@ def forward_backward_loops(X, W, b, Q, shift_labels=None, ignore_index=-100, tem
         db = [0.0] * V
     return dict(loss=loss, dX=np.array(dX), dW=np.array(dW) if compute_dW else None,
                 db=np.array(db) if compute_db else None)
+
+
+def ce_forward_backward(X, W, b, target, ignore_index=-100, temperature=1.0,
+                        reduction="batchmean", compute_dW=True, compute_db=False,
+                        dX_rows=None, dW_rows=None, row_block=256):
+    """Fused linear cross-entropy, fp64: the KL loss above with a one-hot
+    teacher (the cross-entropy of fused_linear_cross_entropy, named on the
+    FusedLinearKLDivLoss page, *Summary*, as the source of its token-chunk
+    geometry).  Written from the cross-entropy definition:
+
+        l_r = lse(u_r) - u_{r, y_r},   u = (X W^T + b) / T,
+        d loss / d z_rv = (p_rv - [v == y_r]) / (T D),
+
+    on rows whose target differs from ignore_index (the target doubles as the
+    row mask); D follows the same reductions as the KL loss (batchmean:
+    N_valid, mean: N_valid * V, sum: 1).  A target outside [0, V) that is not
+    ignore_index makes its row contribute nothing (no teacher mass).
+    """
+    if reduction not in REDUCTIONS:
+        raise OracleError(f"reduction={reduction!r} is not supported")
+    if compute_db and b is None:
+        raise OracleError("compute_db needs a bias")
+    BT, H = np.shape(X)
+    V = np.shape(W)[0]
+    T = float(temperature)
+    tgt = np.asarray(target).astype(np.int64)
+    valid = tgt != np.int64(ignore_index)
+    n_valid = int(valid.sum())
+    D = divisor(reduction, n_valid, V)
+    scale = 0.0 if n_valid == 0 else 1.0 / (T * D)
+    W64 = _as64(W)
+    b64 = _as64(b)
+    dx_sel = np.arange(BT) if dX_rows is None else np.asarray(dX_rows, dtype=np.int64)
+    dw_sel = None if not compute_dW else (np.arange(V) if dW_rows is None
+                                          else np.asarray(dW_rows, dtype=np.int64))
+    dX = np.zeros((len(dx_sel), H))
+    dW = None if dw_sel is None else np.zeros((len(dw_sel), H))
+    db = np.zeros(V) if compute_db else None
+    row_loss = np.zeros(BT)
+    dx_pos = {int(r): i for i, r in enumerate(dx_sel)}
+    for r0 in range(0, BT, row_block):
+        r1 = min(BT, r0 + row_block)
+        Xc = _as64(X[r0:r1])
+        z = Xc @ W64.T
+        if b64 is not None:
+            z += b64
+        u = z / T
+        logp, lse = log_softmax_rows(u)
+        y = tgt[r0:r1]
+        inside = valid[r0:r1] & (y >= 0) & (y < V)
+        rows = np.arange(r1 - r0)
+        ycl = np.clip(y, 0, V - 1)
+        rl = np.where(inside, -logp[rows, ycl], 0.0)
+        row_loss[r0:r1] = rl
+        G = np.exp(logp)
+        G[rows[inside], ycl[inside]] -= 1.0
+        G[~inside] = 0.0
+        G *= scale
+        here = [i for i in range(r0, r1) if i in dx_pos]
+        if here:
+            dX[[dx_pos[i] for i in here]] = G[np.asarray(here) - r0] @ W64
+        if dW is not None:
+            dW += G[:, dw_sel].T @ Xc
+        if db is not None:
+            db += G.sum(axis=0)
+    loss = 0.0 if n_valid == 0 else float(row_loss.sum() / D)
+    return dict(loss=loss, dX=dX, dW=dW, db=db, row_loss=row_loss, n_valid=n_valid, D=D)

@@ -28,6 +28,16 @@ def run_gpu(inp: dict, compute_dW=None, compute_db=None, accum_fp32=None, device
 
     dev = torch.device(device)
     g = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    if g.get("target") is not None:  # cross-entropy workload
+        r = pkg.cross_entropy_forward_backward(
+            g["X"], g["W"], g["b"], g["target"], g["ignore_index"], g["temperature"],
+            g["reduction"],
+            compute_dW=inp["compute_dW"] if compute_dW is None else compute_dW,
+            compute_db=inp["compute_db"] if compute_db is None else compute_db,
+            accum_fp32=inp["accum_fp32"] if accum_fp32 is None else accum_fp32,
+            check_status=True)
+        torch.cuda.synchronize()
+        return r
     r = pkg.forward_backward(
         g["X"], g["W"], g["b"], g["Q"], g["shift_labels"], g["ignore_index"], g["temperature"],
         g["eps"], g["reduction"],
@@ -40,6 +50,14 @@ def run_gpu(inp: dict, compute_dW=None, compute_db=None, accum_fp32=None, device
 
 
 def run_oracle(inp: dict, dX_rows=None, dW_rows=None, compute_dW=None, compute_db=None):
+    if inp.get("target") is not None:
+        from oracle import ce_forward_backward
+        return ce_forward_backward(
+            to_np(inp["X"]), to_np(inp["W"]), to_np(inp["b"]), inp["target"].cpu().numpy(),
+            inp["ignore_index"], inp["temperature"], inp["reduction"],
+            compute_dW=inp["compute_dW"] if compute_dW is None else compute_dW,
+            compute_db=inp["compute_db"] if compute_db is None else compute_db,
+            dX_rows=dX_rows, dW_rows=dW_rows)
     lab = inp["shift_labels"]
     return oracle_fb(
         to_np(inp["X"]), to_np(inp["W"]), to_np(inp["b"]), to_np(inp["Q"]),

@@ -130,3 +130,11 @@ def test_empty_rows_allow_null_row_tensors_but_need_workspace():
 def test_python_module_refuses_reduction_none():
     with pytest.raises(ValueError):
         pkg.FusedLinearKLDivLoss(reduction="none")
+
+
+@no_gpu
+def test_ce_entry_needs_targets():
+    assert pkg.flkl_ce_forward_backward(P, P, None, None, -100, 64, 64, 64, 1, 1.0, 0, 1, 0, 1,
+                                        P, P, P, None, P, 0, None) == INVALID
+    assert pkg.flkl_ce_forward_backward(P, P, None, P, -100, 64, 64, 64, 1, 1.0, 3, 1, 0, 1,
+                                        P, P, P, None, P, 0, None) == UNSUPPORTED

@@ -330,3 +330,59 @@ def test_finite_differences(reduction):
                       - loss(args_m["X"], args_m["W"], args_m["b"])) / (2 * h)
         scale = np.abs(grad).max()
         assert np.abs(num - grad).max() <= 1e-7 * scale + 1e-12, name
+
+
+# ---------------------------------------------------------------- cross-entropy oracle
+
+@pytest.mark.parametrize("reduction", ["batchmean", "sum"])
+@pytest.mark.parametrize("T", [1.0, 1.7])
+def test_ce_oracle_matches_torch_cross_entropy(reduction, T):
+    """torch's cross_entropy with ignore_index (fp64, autograd): its 'mean'
+    divides by the kept rows, which is batchmean here."""
+    from oracle import ce_forward_backward
+    rng = np.random.default_rng(20)
+    X, W, b, _ = _rand_case(rng, BT=8, H=5, V=11)
+    y = rng.integers(0, 11, size=8)
+    y[[2, 5]] = -100
+    r = ce_forward_backward(X, W, b, y, ignore_index=-100, temperature=T, reduction=reduction,
+                            compute_db=True)
+    Xt = torch.tensor(X, requires_grad=True)
+    Wt = torch.tensor(W, requires_grad=True)
+    bt = torch.tensor(b, requires_grad=True)
+    ce = F.cross_entropy(F.linear(Xt, Wt, bt) / T, torch.tensor(y), ignore_index=-100,
+                         reduction="mean" if reduction == "batchmean" else "sum")
+    ce.backward()
+    assert r["loss"] == pytest.approx(ce.item(), rel=1e-13)
+    np.testing.assert_allclose(r["dX"], Xt.grad.numpy(), rtol=1e-11, atol=1e-16)
+    np.testing.assert_allclose(r["dW"], Wt.grad.numpy(), rtol=1e-11, atol=1e-16)
+    np.testing.assert_allclose(r["db"], bt.grad.numpy(), rtol=1e-11, atol=1e-16)
+
+
+@pytest.mark.parametrize("reduction", ["batchmean", "mean", "sum"])
+def test_ce_oracle_is_kl_with_one_hot_teacher(reduction):
+    from oracle import ce_forward_backward
+    rng = np.random.default_rng(21)
+    X, W, b, _ = _rand_case(rng, BT=7, H=4, V=9)
+    y = rng.integers(0, 9, size=7)
+    y[3] = -100
+    Q = np.zeros((7, 9))
+    Q[np.arange(7)[y >= 0], y[y >= 0]] = 1.0
+    a = ce_forward_backward(X, W, b, y, temperature=0.6, reduction=reduction, compute_db=True,
+                            row_block=3)
+    k = forward_backward(X, W, b, Q, shift_labels=y, temperature=0.6, reduction=reduction,
+                         compute_db=True)
+    assert a["loss"] == pytest.approx(k["loss"], rel=1e-13)
+    for key in ("dX", "dW", "db"):
+        np.testing.assert_allclose(a[key], k[key], rtol=1e-12, atol=1e-16)
+
+
+def test_ce_oracle_out_of_range_target_contributes_nothing():
+    from oracle import ce_forward_backward
+    rng = np.random.default_rng(22)
+    X, W, b, _ = _rand_case(rng, BT=4, H=4, V=6)
+    y = np.array([1, 9, 2, -5])
+    r = ce_forward_backward(X, W, b, y, reduction="sum", compute_db=True)
+    keep = ce_forward_backward(X[[0, 2]], W, b, y[[0, 2]], reduction="sum", compute_db=True)
+    assert r["loss"] == pytest.approx(keep["loss"], rel=1e-13)
+    assert np.all(r["dX"][[1, 3]] == 0.0)
+    np.testing.assert_allclose(r["dW"], keep["dW"], rtol=1e-12, atol=1e-16)
