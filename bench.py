@@ -10,8 +10,9 @@ device memory.  Prints one JSON line on rank 0.
 * value      rows (tokens) per second over all ranks, timed with CUDA events
              on the launch stream around exactly K steps (max over ranks);
 * e2e        the same metric through the public Python API with the batch
-             (X, Q, labels) copied from pinned host memory every step and the
-             loss read back to the host every step; the head W stays resident;
+             (X, Q or targets, labels) copied from pinned host memory every
+             step (BatchPipeline: the copy of step i+1 overlaps the loss of
+             step i) and every loss read back; the head W stays resident;
 * roofline   the dominant kernel (largest share of the step's device time)
              from a second, profiled run of K steps: its GEMM FLOPs per launch
              over its average launch time, against the measured bf16 peak;
@@ -366,28 +367,33 @@ def run_ours(args):
                      "peaks": peaks_src}
 
     # ---------------- end to end: batch from pinned host memory, loss back
-    # the step's batch: X, and the teacher Q (or the targets) and the labels
-    batch = [t for t in (X, Q, lab, tgt) if t is not None]
+    # End to end through the public API: every step's batch (X and the
+    # teacher Q, or the targets, and the shift labels) comes from pinned host
+    # memory; BatchPipeline overlaps the copy of step i+1 with the loss of
+    # step i (two device buffers, a copy stream) and reads every loss back.
+    from lm_head_projection_b200.pipeline import BatchPipeline
+
+    batch = [t for t in ((X, tgt) if w.ce else (X, Q, lab)) if t is not None]
     hosts = [t.cpu().pin_memory() for t in batch]
-    hloss = torch.empty((), dtype=torch.float32).pin_memory()
     h2d = sum(h.numel() * h.element_size() for h in hosts)
-
-    def copy_batch():
-        for d, h in zip(batch, hosts):
-            d.copy_(h, non_blocking=True)
-
+    opts = dict(ignore_index=inp["ignore_index"], temperature=inp["temperature"],
+                reduction=inp["reduction"], compute_dW=inp["compute_dW"],
+                compute_db=compute_db, accum_fp32=inp["accum_fp32"])
+    if not w.ce:
+        opts["eps"] = inp["eps"]
+    pipe = BatchPipeline(W, b, kind="ce" if w.ce else "kl", options=opts,
+                         compute_stream=stream, max_steps=args.steps + args.warmup + 4)
     for _ in range(max(1, args.warmup)):
-        copy_batch()
-        api_call(out=out, workspace=ws)
-        hloss.copy_(out["loss"], non_blocking=True)
+        pipe.submit(hosts)
+    pipe.finish()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     e0.record(stream)
+    pipe.copy.wait_event(e0)
     for _ in range(args.steps):
-        copy_batch()
-        api_call(out=out, workspace=ws)
-        hloss.copy_(out["loss"], non_blocking=True)
+        pipe.submit(hosts)
+    pipe.finish()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -257,3 +257,37 @@ def test_profiled_entry_records_every_launch_and_matches():
         assert events[2 * i].elapsed_time(events[2 * i + 1]) >= 0.0
     for k in ("loss", "dX", "dW", "db"):
         assert torch.equal(out[k], ref[k]), k
+
+
+def test_batch_pipeline_matches_direct_calls():
+    """The double-buffered host-batch pipeline gives, step by step, the loss
+    of direct calls on the same batches, for the KL and the CE losses."""
+    from lm_head_projection_b200.pipeline import BatchPipeline
+
+    dev = torch.device("cuda:0")
+    for ce in (False, True):
+        ws = [small_case(dtype="bf16", BT=96, H=128, V=1000, bias=True, ce=ce, ignore_frac=0.1,
+                         seed=s) for s in (1, 2, 3)]
+        inps = [make_inputs(w) for w in ws]
+        W = inps[0]["W"].to(dev)
+        b = inps[0]["b"].to(dev)
+        opts = dict(ignore_index=-100, temperature=1.0, reduction="batchmean",
+                    compute_dW=True, compute_db=True, accum_fp32=True)
+        if not ce:
+            opts["eps"] = 1e-10
+        pipe = BatchPipeline(W, b, kind="ce" if ce else "kl", options=opts)
+        direct = []
+        for inp in inps:
+            host = ([inp["X"].pin_memory(), inp["target"].pin_memory()] if ce else
+                    [inp["X"].pin_memory(), inp["Q"].pin_memory(),
+                     inp["shift_labels"].pin_memory()])
+            pipe.submit(host)
+            d = dict(inp, W=inps[0]["W"], b=inps[0]["b"])
+            direct.append(float(run_gpu(d)["loss"].cpu()))
+        pipe.finish()
+        torch.cuda.synchronize()
+        got = pipe.losses().tolist()
+        assert got == direct, (ce, got, direct)
+        last = run_gpu(dict(inps[-1], W=inps[0]["W"], b=inps[0]["b"]))
+        assert torch.equal(pipe.out["dX"], last["dX"])
+        assert torch.equal(pipe.out["dW"], last["dW"])
