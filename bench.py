@@ -101,6 +101,12 @@ def parse():
     ap.add_argument("--cpu-sample-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="loss", choices=["loss", "rms_norm", "layer_norm"],
+                    help="loss: the fused linear KL / CE loss (default); rms_norm / "
+                         "layer_norm: the norm backward with frozen-parameter flags")
+    ap.add_argument("--norm-shape", default="8192x8192", help="ROWSxH for --op *_norm")
+    ap.add_argument("--norm-dtype", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--frozen", action="store_true", help="norm weight (and bias) frozen")
     return ap.parse_args()
 
 
@@ -478,9 +484,86 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_norm(args):
+    """Norm backward on one GPU: device time of each launch (CUDA events on the
+    launching stream), with L2 flushed between launches outside the events."""
+    import numpy as np
+
+    from lm_head_projection_b200 import norm
+    from lm_head_projection_b200.workloads import make_norm_inputs
+
+    rows, H = (int(v) for v in args.norm_shape.lower().split("x"))
+    layer = args.op == "layer_norm"
+    train = not args.frozen
+    dev = torch.device("cuda", 0)
+    inp = {k: v.to(dev) for k, v in make_norm_inputs(rows, H, args.norm_dtype, 0).items()}
+    e = 4 if args.norm_dtype == "fp32" else 2
+
+    def step():
+        if layer:
+            return norm.layer_norm_backward(inp["dY"], inp["X"], inp["W"], compute_dW=train,
+                                            compute_db=train)
+        return norm.rms_norm_backward(inp["dY"], inp["X"], inp["W"], compute_dW=train)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    med = ms[len(ms) // 2]
+    n_grads = (2 if layer else 1) if train else 0
+    algo = 3 * rows * H * e + H * e + n_grads * H * 4
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("hbm_gbs")
+    achieved = algo / (med * 1e-3) / 1e9
+    # the oracle on the host cores, the same shape
+    from oracle.norm_oracle import layer_norm_backward as o_ln
+    from oracle.norm_oracle import rms_norm_backward as o_rms
+    host = {k: v.float().cpu().numpy().astype(np.float64) for k, v in inp.items()}
+    t0 = time.perf_counter()
+    if layer:
+        o_ln(host["dY"], host["X"], host["W"], 1e-5, train, train)
+    else:
+        o_rms(host["dY"], host["X"], host["W"], 1e-6, train)
+    t_cpu = time.perf_counter() - t0
+    name = f"{args.op}_{args.norm_dtype}_{rows}x{H}{'_frozen' if args.frozen else ''}"
+    line = {
+        "metric": "norm_backward_rows_per_s", "value": round(rows / (med * 1e-3), 1),
+        "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(med, 5), "ms_min": round(ms[0], 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if args.norm_dtype == "fp32" else "bf16", "data": "synthetic",
+        "config": {"workload": name, "rows": rows, "H": H, "l2": "flushed between launches"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4) if peak else None,
+                     "traffic": None, "algorithmic_bytes": algo, "peak_source": peak_src},
+        "cpu_baseline": {"value": round(rows / t_cpu, 1), "unit": "rows/s",
+                         "cores": host_threads(), "kind": "oracle",
+                         "sample": f"the whole {rows}x{H} problem once, fp64 numpy"},
+        "clocks": clocks.summary(),
+        "gpu_launches": args.steps * (1 + n_grads),
+    }
+    print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.impl == "reference":
+    if a.op != "loss":
+        run_norm(a)
+    elif a.impl == "reference":
         run_reference(a)
     else:
         run_ours(a)

@@ -219,6 +219,42 @@ FLKL_API flkl_status flkl_forward_backward_noalloc(
     float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
     void* dX, void* dW, void* db, void* stream);
 
+/* RMSNorm / LayerNorm backward with frozen-parameter flags (the LoRA
+ * normalization pull-request page, Key Changes: COMPUTE_DW for RMSNorm,
+ * COMPUTE_DW / COMPUTE_DB for LayerNorm; with a frozen parameter its gradient
+ * is neither accumulated nor reduced and dX is unchanged).
+ *
+ *   RMSNorm:   y = w * x / sqrt(mean(x^2) + eps)
+ *   LayerNorm: y = w * (x - mean(x)) / sqrt(var(x) + eps) + b  (biased var)
+ *
+ * over the last dimension of x [rows, H], for the incoming gradient dY
+ * [rows, H]; the row statistics are recomputed from X.
+ *
+ *  dY, X, W     device; dY and X [rows, H], W [H]; all `dtype`.
+ *  rows, H      rows >= 0; 1 <= H <= 8192 and H a multiple of 8.
+ *  eps          >= 0.
+ *  compute_dW   nonzero: write dW [H] (dW non-NULL), else dW must be NULL.
+ *  compute_db   (LayerNorm) nonzero: write db [H] = sum of dY over rows.
+ *  accum_fp32   nonzero: dW / db are fp32, else `dtype`.
+ *  dX           device [rows, H], `dtype` (overwritten).
+ *  workspace    device, flkl_norm_workspace_size(...) bytes, 256-byte aligned
+ *               (may be NULL when that size is 0, i.e. both flags are 0).
+ *  Pointers 16-byte aligned (else FLKL_ERR_UNSUPPORTED).  Asynchronous on
+ *  `stream`; errors as flkl_forward_backward.  Deterministic: dW and db are
+ *  summed in a fixed order that does not depend on the device. */
+FLKL_API size_t flkl_norm_workspace_size(int64_t rows, int64_t H, int compute_dW,
+                                         int compute_db);
+FLKL_API flkl_status flkl_rms_norm_backward(const void* dY, const void* X, const void* W,
+                                            int64_t rows, int64_t H, int dtype, float eps,
+                                            int compute_dW, int accum_fp32, void* dX, void* dW,
+                                            void* workspace, size_t workspace_bytes,
+                                            void* stream);
+FLKL_API flkl_status flkl_layer_norm_backward(const void* dY, const void* X, const void* W,
+                                              int64_t rows, int64_t H, int dtype, float eps,
+                                              int compute_dW, int compute_db, int accum_fp32,
+                                              void* dX, void* dW, void* db, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device status recorded by the last
  * flkl_forward_backward call that used `workspace` (FLKL_OK or
  * FLKL_ERR_TIMEOUT), or FLKL_ERR_CUDA if the copy or the synchronisation

@@ -21,6 +21,7 @@ __all__ = [
     "flkl_device_status", "flkl_set_wait_limit_ms", "flkl_wait_selftest", "flkl_status_string",
     "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
     "flkl_ce_forward_backward", "cross_entropy_forward_backward", "FusedLinearCrossEntropyLoss",
+    "flkl_norm_workspace_size", "flkl_rms_norm_backward", "flkl_layer_norm_backward",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +89,17 @@ def _lib():
         lib.flkl_wait_selftest.argtypes = [c.c_void_p, c.c_uint, c.c_void_p]
         lib.flkl_status_string.restype = c.c_char_p
         lib.flkl_status_string.argtypes = [c.c_int]
+        lib.flkl_norm_workspace_size.restype = c.c_size_t
+        lib.flkl_norm_workspace_size.argtypes = [c.c_int64, c.c_int64, c.c_int, c.c_int]
+        lib.flkl_rms_norm_backward.restype = c.c_int
+        lib.flkl_rms_norm_backward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int, c.c_float,
+            c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.flkl_layer_norm_backward.restype = c.c_int
+        lib.flkl_layer_norm_backward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int, c.c_float,
+            c.c_int, c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+            c.c_size_t, c.c_void_p]
         _LIB = lib
     return _LIB
 
@@ -127,6 +139,28 @@ def flkl_ce_forward_backward(X, W, b, target, ignore_index, BT, H, V, dtype, tem
         X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
         float(temperature), int(reduction), int(bool(compute_dW)), int(bool(compute_db)),
         int(bool(accum_fp32)), loss, dX, dW, db, workspace, int(workspace_bytes), stream)
+
+
+def flkl_norm_workspace_size(rows, H, compute_dW, compute_db) -> int:
+    return _lib().flkl_norm_workspace_size(int(rows), int(H), int(bool(compute_dW)),
+                                           int(bool(compute_db)))
+
+
+def flkl_rms_norm_backward(dY, X, W, rows, H, dtype, eps, compute_dW, accum_fp32, dX, dW,
+                           workspace, workspace_bytes, stream) -> int:
+    """The RMSNorm-backward C entry point with raw pointers; returns the status."""
+    return _lib().flkl_rms_norm_backward(
+        dY, X, W, int(rows), int(H), int(dtype), float(eps), int(bool(compute_dW)),
+        int(bool(accum_fp32)), dX, dW, workspace, int(workspace_bytes), stream)
+
+
+def flkl_layer_norm_backward(dY, X, W, rows, H, dtype, eps, compute_dW, compute_db, accum_fp32,
+                             dX, dW, db, workspace, workspace_bytes, stream) -> int:
+    """The LayerNorm-backward C entry point with raw pointers; returns the status."""
+    return _lib().flkl_layer_norm_backward(
+        dY, X, W, int(rows), int(H), int(dtype), float(eps), int(bool(compute_dW)),
+        int(bool(compute_db)), int(bool(accum_fp32)), dX, dW, db, workspace,
+        int(workspace_bytes), stream)
 
 
 def flkl_forward_backward_noalloc(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,

@@ -14,8 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "_flkl.so")
-SOURCES = ["flkl_api.cu"]
-HEADERS = ["ptx.cuh", "tc_gemm.cuh", "row_kernels.cuh", "simt_f32.cuh"]
+SOURCES = ["flkl_api.cu", "norm_api.cu"]
+HEADERS = ["ptx.cuh", "tc_gemm.cuh", "row_kernels.cuh", "simt_f32.cuh", "norm_bwd.cuh"]
 
 
 def nvcc_path() -> str:

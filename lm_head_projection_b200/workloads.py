@@ -211,3 +211,24 @@ def small_case(dtype="bf16", BT=133, H=192, V=1000, bias=True, reduction="batchm
     return Workload(f"small_{'ce_' if ce else ''}{dtype}_{BT}x{H}x{V}", dtype, BT, H, V, bias,
                     x_std, w_std, b_std, q_std, temperature, eps, reduction, compute_dW,
                     compute_db, True, ignore_frac, zero_frac, seed, ce)
+
+
+# ----------------------------------------------------------------- norm backward
+# Shapes (rows, H) of the LoRA normalization pull-request page, *Benchmark
+# Results* (bf16).  That page names no input distribution; the one below is a
+# plain choice: hidden states with a per-row offset (so LayerNorm's centring
+# matters), a unit-scale incoming gradient, and norm weights near 1.
+NORM_SHAPES = [(2048, 4096), (4096, 4096), (4096, 8192), (8192, 4096), (8192, 8192)]
+_S_NX, _S_NXM, _S_NDY, _S_NW = range(11, 15)
+
+
+def make_norm_inputs(rows: int, H: int, dtype: str = "bf16", seed: int = 0,
+                     device="cpu") -> dict:
+    """dY, X [rows, H] and W [H]: X = m_row + N(0, 1) with m_row ~ N(0, 1),
+    dY ~ N(0, 1), W = 1 + N(0, 0.1^2); cast to ``dtype`` ("fp32" | "bf16")."""
+    dt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    x = torch.randn((rows, H), generator=_gen(device, seed, _S_NX), device=device)
+    x += torch.randn((rows, 1), generator=_gen(device, seed, _S_NXM), device=device)
+    dy = torch.randn((rows, H), generator=_gen(device, seed, _S_NDY), device=device)
+    w = 1.0 + 0.1 * torch.randn((H,), generator=_gen(device, seed, _S_NW), device=device)
+    return dict(dY=dy.to(dt), X=x.to(dt), W=w.to(dt))

@@ -138,3 +138,57 @@ def test_ce_entry_needs_targets():
                                         P, P, P, None, P, 0, None) == INVALID
     assert pkg.flkl_ce_forward_backward(P, P, None, P, -100, 64, 64, 64, 1, 1.0, 3, 1, 0, 1,
                                         P, P, P, None, P, 0, None) == UNSUPPORTED
+
+
+def norm_call(layer=False, **kw):
+    a = dict(dY=P, X=P, W=P, rows=64, H=4096, dtype=1, eps=1e-6, compute_dW=1, compute_db=0,
+             accum_fp32=1, dX=P, dW=P, db=None, workspace=P, workspace_bytes=1 << 30,
+             stream=None)
+    a.update(kw)
+    if layer:
+        return pkg.flkl_layer_norm_backward(**a)
+    a.pop("compute_db"), a.pop("db")
+    return pkg.flkl_rms_norm_backward(**a)
+
+
+def test_norm_workspace_size_rules():
+    # one fp32 partial row per block and per gradient asked for; nothing when frozen
+    assert pkg.flkl_norm_workspace_size(8192, 4096, 0, 0) == 0
+    one = pkg.flkl_norm_workspace_size(8192, 4096, 1, 0)
+    assert one == pkg.flkl_norm_workspace_size(8192, 4096, 0, 1) > 0
+    assert pkg.flkl_norm_workspace_size(8192, 4096, 1, 1) == 2 * one
+    assert one % 256 == 0 and one < 8192 * 4096 * 4 // 8
+    assert pkg.flkl_norm_workspace_size(3, 64, 1, 0) == 3 * 64 * 4   # 3 rows -> 3 blocks
+    assert pkg.flkl_norm_workspace_size(10, 8200, 1, 0) == 0  # H above the limit
+
+
+@no_gpu
+@pytest.mark.parametrize("layer", [False, True])
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dtype=4), INVALID),
+    (dict(rows=-1), INVALID),
+    (dict(H=0), INVALID),
+    (dict(eps=-1.0), INVALID),
+    (dict(eps=float("nan")), INVALID),
+    (dict(H=4100), UNSUPPORTED),                # not a multiple of 8
+    (dict(H=8200), UNSUPPORTED),                # above 8192
+    (dict(W=None), INVALID),
+    (dict(X=None), INVALID),
+    (dict(dY=None), INVALID),
+    (dict(dX=None), INVALID),
+    (dict(dW=None), INVALID),                   # compute_dW without dW
+    (dict(compute_dW=0), INVALID),              # dW given while frozen
+    (dict(X=P + 8), UNSUPPORTED),
+    (dict(dW=P + 4), UNSUPPORTED),
+    (dict(workspace=None), WORKSPACE),
+    (dict(workspace=P + 16), WORKSPACE),        # not 256-aligned
+    (dict(workspace_bytes=100), WORKSPACE),
+])
+def test_norm_host_rejects_bad_arguments(layer, kw, expect):
+    assert norm_call(layer, **kw) == expect
+
+
+@no_gpu
+def test_layer_norm_bias_flag_needs_pointer():
+    assert norm_call(True, compute_db=1) == INVALID            # db missing
+    assert norm_call(True, compute_db=0, db=P) == INVALID      # db not asked for
