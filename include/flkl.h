@@ -147,6 +147,10 @@ FLKL_API flkl_status flkl_ce_forward_backward(const void* X, const void* W, cons
                                               int compute_db, int accum_fp32, float* loss,
                                               void* dX, void* dW, void* db, void* workspace,
                                               size_t workspace_bytes, void* stream);
+/* Synchronises `stream` and returns the status word of the norm-backward
+ * kernels of the current device (FLKL_OK, or FLKL_ERR_TIMEOUT when one of
+ * their waits gave up since the last call), then clears it. */
+FLKL_API flkl_status flkl_norm_device_status(void* stream);
 
 /* Kinds of launches reported by flkl_forward_backward_profiled. */
 typedef enum {
@@ -240,8 +244,12 @@ FLKL_API flkl_status flkl_forward_backward_noalloc(
  *  workspace    device, flkl_norm_workspace_size(...) bytes, 256-byte aligned
  *               (may be NULL when that size is 0, i.e. both flags are 0).
  *  Pointers 16-byte aligned (else FLKL_ERR_UNSUPPORTED).  Asynchronous on
- *  `stream`; errors as flkl_forward_backward.  Deterministic: dW and db are
- *  summed in a fixed order that does not depend on the device. */
+ *  `stream`; host-side errors as flkl_forward_backward.  A device-side wait
+ *  that gives up (flkl_set_wait_limit_ms) leaves dX undefined and is reported
+ *  by flkl_norm_device_status.  Deterministic on a given device: dW and db
+ *  are summed in a fixed order (per-CTA partial rows, then in CTA order).
+ *  The workspace holds one fp32 partial row of H per CTA and per gradient
+ *  asked for; its size depends on the current device's SM count. */
 FLKL_API size_t flkl_norm_workspace_size(int64_t rows, int64_t H, int compute_dW,
                                          int compute_db);
 FLKL_API flkl_status flkl_rms_norm_backward(const void* dY, const void* X, const void* W,

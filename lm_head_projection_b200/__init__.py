@@ -22,6 +22,7 @@ __all__ = [
     "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
     "flkl_ce_forward_backward", "cross_entropy_forward_backward", "FusedLinearCrossEntropyLoss",
     "flkl_norm_workspace_size", "flkl_rms_norm_backward", "flkl_layer_norm_backward",
+    "flkl_norm_device_status",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +96,8 @@ def _lib():
         lib.flkl_rms_norm_backward.argtypes = [
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int, c.c_float,
             c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.flkl_norm_device_status.restype = c.c_int
+        lib.flkl_norm_device_status.argtypes = [c.c_void_p]
         lib.flkl_layer_norm_backward.restype = c.c_int
         lib.flkl_layer_norm_backward.argtypes = [
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int, c.c_float,
@@ -161,6 +164,11 @@ def flkl_layer_norm_backward(dY, X, W, rows, H, dtype, eps, compute_dW, compute_
         dY, X, W, int(rows), int(H), int(dtype), float(eps), int(bool(compute_dW)),
         int(bool(compute_db)), int(bool(accum_fp32)), dX, dW, db, workspace,
         int(workspace_bytes), stream)
+
+
+def flkl_norm_device_status(stream=None) -> int:
+    """Synchronise ``stream``; status of the norm kernels since the last call."""
+    return _lib().flkl_norm_device_status(stream)
 
 
 def flkl_forward_backward_noalloc(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,

@@ -26,12 +26,14 @@
 #include "tc_gemm.cuh"
 
 namespace flkl {
+
+// Limit of every bounded wait in the library's kernels (flkl_set_wait_limit_ms).
+unsigned long long g_wait_limit_ns = 4000ull * 1000000ull;
+
 namespace {
 
 constexpr size_t kStagingBudget = size_t(256) << 20;  // bytes of G staging at most
 constexpr int kMaxDevices = 64;
-
-unsigned long long g_wait_limit_ns = 4000ull * 1000000ull;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 long long cdiv(long long a, long long b) { return (a + b - 1) / b; }

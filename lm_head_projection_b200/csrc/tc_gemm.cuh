@@ -115,17 +115,6 @@ __device__ __forceinline__ DescSteps desc_steps(bool mn_major) {
   return r;
 }
 
-// Wait (bounded, no abort check) for phase `parity` of a local barrier; used
-// only on exit paths.
-__device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity,
-                                                unsigned long long limit_ns) {
-  const uint32_t addr = smem_u32(bar);
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(addr, parity)) {
-    if (globaltimer_ns() - t0 > limit_ns) break;
-  }
-}
-
 // ====================================================================
 // Epilogues.  `run` is called by each epilogue warp for its 32 rows and 128
 // columns of the tile: lane i owns output row (row0 + quad*32 + i), columns

@@ -157,8 +157,11 @@ def test_norm_workspace_size_rules():
     one = pkg.flkl_norm_workspace_size(8192, 4096, 1, 0)
     assert one == pkg.flkl_norm_workspace_size(8192, 4096, 0, 1) > 0
     assert pkg.flkl_norm_workspace_size(8192, 4096, 1, 1) == 2 * one
-    assert one % 256 == 0 and one < 8192 * 4096 * 4 // 8
-    assert pkg.flkl_norm_workspace_size(3, 64, 1, 0) == 3 * 64 * 4   # 3 rows -> 3 blocks
+    # one fp32 row per CTA, at least 8 rows per CTA, at most 16 CTAs per SM
+    assert one % 256 == 0 and one <= 8192 // 8 * 4096 * 4
+    big = pkg.flkl_norm_workspace_size(1 << 22, 4096, 1, 0)
+    assert big == pkg.flkl_norm_workspace_size(1 << 23, 4096, 1, 0) <= 148 * 16 * 4096 * 4
+    assert pkg.flkl_norm_workspace_size(3, 64, 1, 0) == 256   # 3 rows -> 1 CTA
     assert pkg.flkl_norm_workspace_size(10, 8200, 1, 0) == 0  # H above the limit
 
 

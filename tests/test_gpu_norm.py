@@ -137,6 +137,9 @@ def test_deterministic_parameter_gradients():
     a = norm.layer_norm_backward(inp["dY"], inp["X"], inp["W"])
     b = norm.layer_norm_backward(inp["dY"], inp["X"], inp["W"])
     assert torch.equal(a["dW"], b["dW"]) and torch.equal(a["db"], b["db"])
+    assert torch.equal(a["dX"], b["dX"])
+    import lm_head_projection_b200 as pkg
+    assert pkg.flkl_norm_device_status(torch.cuda.current_stream().cuda_stream) == 0
 
 
 @pytest.mark.parametrize("freeze_w,freeze_b", [(False, False), (True, False), (True, True)])
