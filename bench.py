@@ -58,16 +58,18 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+GEMM_SOURCES = ("flkl_api.cu", "ptx.cuh", "row_kernels.cuh", "tc_gemm.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources the GEMM kernel is built from."""
+    """Hash of the CUDA sources the fused-loss kernels are built from."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "lm_head_projection_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + b"\0" + f.read())
+    for fn in GEMM_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -107,6 +109,9 @@ def parse():
     ap.add_argument("--norm-shape", default="8192x8192", help="ROWSxH for --op *_norm")
     ap.add_argument("--norm-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--frozen", action="store_true", help="norm weight (and bias) frozen")
+    ap.add_argument("--dp", action="store_true",
+                    help="data-parallel training step: whole-batch kept-row count and "
+                         "all-reduce of loss, dW, db (NCCL) inside each timed step")
     return ap.parse_args()
 
 
@@ -278,9 +283,26 @@ def run_ours(args):
                compute_db, inp["accum_fp32"], p(out["loss"]), p(out["dX"]), p(out["dW"]),
                p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
 
+    n_total = torch.zeros((), dtype=torch.int64, device=dev)
+    mask = tgt if w.ce else lab
+    exchanged = [t for t in (out["loss"], out["dW"], out["db"]) if t is not None]
+
     def step():
-        s = (pkg.flkl_ce_forward_backward(*ce_args) if w.ce
-             else pkg.flkl_forward_backward(*call_args))
+        if not args.dp:
+            s = (pkg.flkl_ce_forward_backward(*ce_args) if w.ce
+                 else pkg.flkl_forward_backward(*call_args))
+        else:
+            # the data-parallel step of lm_head_projection_b200.dp, raw entry points
+            s = pkg.flkl_count_valid(p(mask), w.BT, inp["ignore_index"], p(n_total),
+                                     stream.cuda_stream)
+            if s == 0:
+                if world > 1:
+                    dist.all_reduce(n_total)
+                s = (pkg.flkl_ce_forward_backward_dp(*ce_args, p(n_total)) if w.ce
+                     else pkg.flkl_forward_backward_dp(*call_args, p(n_total)))
+            if s == 0 and world > 1:
+                for t in exchanged:
+                    dist.all_reduce(t)
         if s != 0:
             raise pkg.FlklError(s, "flkl_forward_backward")
 
@@ -426,10 +448,12 @@ def run_ours(args):
             "config": {"workload": w.name, "global_batch": w.BT * world, "BT_per_gpu": w.BT,
                        "H": w.H, "V": w.V, "compute_dW": w.compute_dW,
                        "compute_db": bool(compute_db), "reduction": w.reduction,
-                       "temperature": w.temperature, "parallelism": f"dp{world}",
+                       "temperature": w.temperature,
+                       "parallelism": f"dp{world}" + ("-allreduce" if args.dp else "-replicas"),
                        "l2": "inputs larger than L2 (W, Q), no flush"},
             "e2e": e2e, "roofline": roofline, "step_roofline": step_roofline,
-            "kernels": breakdown, "gpu_launches": int(launches_per_step * args.steps),
+            "kernels": breakdown,
+            "gpu_launches": int((launches_per_step + (1 if args.dp else 0)) * args.steps),
             "clocks": clk, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

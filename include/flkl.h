@@ -147,10 +147,33 @@ FLKL_API flkl_status flkl_ce_forward_backward(const void* X, const void* W, cons
                                               int compute_db, int accum_fp32, float* loss,
                                               void* dX, void* dW, void* db, void* workspace,
                                               size_t workspace_bytes, void* stream);
-/* Synchronises `stream` and returns the status word of the norm-backward
- * kernels of the current device (FLKL_OK, or FLKL_ERR_TIMEOUT when one of
- * their waits gave up since the last call), then clears it. */
-FLKL_API flkl_status flkl_norm_device_status(void* stream);
+
+/* Data-parallel use: the batch is split by rows over ranks that share the
+ * head W, b (the row sharding of the scope table's multi-GPU row).  Each rank
+ * calls flkl_count_valid on its labels (or targets), all-reduces the int64
+ * count (sum) into `n_valid_total`, calls the _dp entry below, then
+ * all-reduces loss, dW and db (sum); dX needs no exchange.  The _dp entries
+ * are flkl_forward_backward / flkl_ce_forward_backward with the divisor of
+ * the reduction taken from *n_valid_total (device int64, 8-byte aligned,
+ * read on the device, non-NULL) instead of this call's kept rows, so the
+ * per-rank results add up to the whole batch's.  No collective runs in the
+ * library.
+ *
+ * flkl_count_valid: *count (device int64) = rows r < BT with labels[r] !=
+ * ignore_index (labels NULL: BT).  Asynchronous on `stream`. */
+FLKL_API flkl_status flkl_count_valid(const int64_t* labels, int64_t BT, int64_t ignore_index,
+                                      int64_t* count, void* stream);
+FLKL_API flkl_status flkl_forward_backward_dp(
+    const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
+    int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
+    float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
+    void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
+    const int64_t* n_valid_total);
+FLKL_API flkl_status flkl_ce_forward_backward_dp(
+    const void* X, const void* W, const void* b, const int64_t* target, int64_t ignore_index,
+    int64_t BT, int64_t H, int64_t V, int dtype, float temperature, int reduction,
+    int compute_dW, int compute_db, int accum_fp32, float* loss, void* dX, void* dW, void* db,
+    void* workspace, size_t workspace_bytes, void* stream, const int64_t* n_valid_total);
 
 /* Kinds of launches reported by flkl_forward_backward_profiled. */
 typedef enum {
@@ -262,6 +285,10 @@ FLKL_API flkl_status flkl_layer_norm_backward(const void* dY, const void* X, con
                                               int compute_dW, int compute_db, int accum_fp32,
                                               void* dX, void* dW, void* db, void* workspace,
                                               size_t workspace_bytes, void* stream);
+/* Synchronises `stream` and returns the status word of the norm-backward
+ * kernels of the current device (FLKL_OK, or FLKL_ERR_TIMEOUT when one of
+ * their waits gave up since the last call), then clears it. */
+FLKL_API flkl_status flkl_norm_device_status(void* stream);
 
 /* Synchronises `stream`, then returns the device status recorded by the last
  * flkl_forward_backward call that used `workspace` (FLKL_OK or

@@ -22,7 +22,8 @@ __all__ = [
     "forward_backward", "FusedLinearKLDivLoss", "library_path", "REDUCTIONS",
     "flkl_ce_forward_backward", "cross_entropy_forward_backward", "FusedLinearCrossEntropyLoss",
     "flkl_norm_workspace_size", "flkl_rms_norm_backward", "flkl_layer_norm_backward",
-    "flkl_norm_device_status",
+    "flkl_norm_device_status", "flkl_count_valid", "flkl_forward_backward_dp",
+    "flkl_ce_forward_backward_dp", "count_valid",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -79,6 +80,14 @@ def _lib():
             c.c_int, c.c_int, c.c_int,                           # dW db accum_fp32
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,      # loss dX dW db
             c.c_void_p, c.c_size_t, c.c_void_p]                  # ws bytes stream
+        lib.flkl_forward_backward_dp.restype = c.c_int
+        lib.flkl_forward_backward_dp.argtypes = list(lib.flkl_forward_backward.argtypes) + [
+            c.c_void_p]
+        lib.flkl_ce_forward_backward_dp.restype = c.c_int
+        lib.flkl_ce_forward_backward_dp.argtypes = list(
+            lib.flkl_ce_forward_backward.argtypes) + [c.c_void_p]
+        lib.flkl_count_valid.restype = c.c_int
+        lib.flkl_count_valid.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p]
         lib.flkl_forward_backward_noalloc.restype = c.c_int
         lib.flkl_forward_backward_noalloc.argtypes = (
             list(lib.flkl_forward_backward.argtypes[:20]) + [c.c_void_p])
@@ -142,6 +151,35 @@ def flkl_ce_forward_backward(X, W, b, target, ignore_index, BT, H, V, dtype, tem
         X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
         float(temperature), int(reduction), int(bool(compute_dW)), int(bool(compute_db)),
         int(bool(accum_fp32)), loss, dX, dW, db, workspace, int(workspace_bytes), stream)
+
+
+def flkl_count_valid(labels, BT, ignore_index, count, stream) -> int:
+    """Kept rows of a batch into the device int64 at ``count``; returns the status."""
+    return _lib().flkl_count_valid(labels, int(BT), int(ignore_index), count, stream)
+
+
+def flkl_forward_backward_dp(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                             temperature, eps, reduction, compute_dW, compute_db, accum_fp32, loss,
+                             dX, dW, db, workspace, workspace_bytes, stream,
+                             n_valid_total) -> int:
+    """flkl_forward_backward with the divisor taken from the device int64 at
+    ``n_valid_total`` (the kept rows of every rank's batch)."""
+    return _lib().flkl_forward_backward_dp(
+        X, W, b, Q, shift_labels, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), float(eps), int(reduction), int(bool(compute_dW)),
+        int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
+        int(workspace_bytes), stream, n_valid_total)
+
+
+def flkl_ce_forward_backward_dp(X, W, b, target, ignore_index, BT, H, V, dtype, temperature,
+                                reduction, compute_dW, compute_db, accum_fp32, loss, dX, dW, db,
+                                workspace, workspace_bytes, stream, n_valid_total) -> int:
+    """flkl_ce_forward_backward with the divisor from ``n_valid_total``."""
+    return _lib().flkl_ce_forward_backward_dp(
+        X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), int(reduction), int(bool(compute_dW)), int(bool(compute_db)),
+        int(bool(accum_fp32)), loss, dX, dW, db, workspace, int(workspace_bytes), stream,
+        n_valid_total)
 
 
 def flkl_norm_workspace_size(rows, H, compute_dW, compute_db) -> int:
@@ -243,12 +281,15 @@ def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
                      temperature: float = 1.0, eps: float = 1e-10, reduction: str = "batchmean",
                      compute_dW: bool = True, compute_db: bool = False, accum_fp32: bool = True,
                      out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
-                     stream: Optional[torch.cuda.Stream] = None, check_status: bool = False) -> dict:
+                     stream: Optional[torch.cuda.Stream] = None, check_status: bool = False,
+                     n_valid_total: Optional[torch.Tensor] = None) -> dict:
     """Loss and gradients in one call on the current CUDA stream.
 
     Allocates outputs (and the workspace) with torch unless given in ``out`` /
     ``workspace``; returns ``{"loss", "dX", "dW", "db"}`` (None for the ones
-    not asked for).  Raises FlklError on a non-OK status.
+    not asked for).  Raises FlklError on a non-OK status.  ``n_valid_total``
+    (a device int64 scalar) replaces the batch's kept-row count in the
+    divisor: the data-parallel form (see :mod:`.dp`).
     """
     if reduction not in REDUCTIONS:
         raise ValueError(f"unknown reduction {reduction!r}")
@@ -286,11 +327,15 @@ def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    status = flkl_forward_backward(
-        _ptr(X), _ptr(W), _ptr(b), _ptr(Q), _ptr(shift_labels), ignore_index, BT, H, V,
-        DTYPES[dt], temperature, eps, REDUCTIONS[reduction], compute_dW, compute_db, accum_fp32,
-        _ptr(loss), _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace), workspace.numel(),
-        st.cuda_stream)
+    args = (_ptr(X), _ptr(W), _ptr(b), _ptr(Q), _ptr(shift_labels), ignore_index, BT, H, V,
+            DTYPES[dt], temperature, eps, REDUCTIONS[reduction], compute_dW, compute_db,
+            accum_fp32, _ptr(loss), _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace),
+            workspace.numel(), st.cuda_stream)
+    if n_valid_total is not None:
+        _check_dev("n_valid_total", n_valid_total, torch.int64, (), dev)
+        status = flkl_forward_backward_dp(*args, _ptr(n_valid_total))
+    else:
+        status = flkl_forward_backward(*args)
     if status != FLKL_OK:
         raise FlklError(status, "flkl_forward_backward")
     if check_status:
@@ -369,7 +414,8 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
                                    accum_fp32: bool = True, out: Optional[dict] = None,
                                    workspace: Optional[torch.Tensor] = None,
                                    stream: Optional[torch.cuda.Stream] = None,
-                                   check_status: bool = False) -> dict:
+                                   check_status: bool = False,
+                                   n_valid_total: Optional[torch.Tensor] = None) -> dict:
     """Fused linear + cross-entropy (one-hot teacher at ``target``) in one call.
     ``reduction="batchmean"`` divides by the kept rows (torch's cross_entropy
     "mean").  Same outputs and conventions as :func:`forward_backward`."""
@@ -407,10 +453,14 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
-    status = flkl_ce_forward_backward(
-        _ptr(X), _ptr(W), _ptr(b), _ptr(target), ignore_index, BT, H, V, DTYPES[dt],
-        temperature, REDUCTIONS[reduction], compute_dW, compute_db, accum_fp32, _ptr(loss),
-        _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace), workspace.numel(), st.cuda_stream)
+    args = (_ptr(X), _ptr(W), _ptr(b), _ptr(target), ignore_index, BT, H, V, DTYPES[dt],
+            temperature, REDUCTIONS[reduction], compute_dW, compute_db, accum_fp32, _ptr(loss),
+            _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace), workspace.numel(), st.cuda_stream)
+    if n_valid_total is not None:
+        _check_dev("n_valid_total", n_valid_total, torch.int64, (), dev)
+        status = flkl_ce_forward_backward_dp(*args, _ptr(n_valid_total))
+    else:
+        status = flkl_ce_forward_backward(*args)
     if status != FLKL_OK:
         raise FlklError(status, "flkl_ce_forward_backward")
     if check_status:
@@ -418,6 +468,22 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
         if s != FLKL_OK:
             raise FlklError(s, "flkl_ce_forward_backward (device)")
     return {"loss": loss, "dX": dX, "dW": dW, "db": db, "workspace": workspace}
+
+
+def count_valid(labels: Optional[torch.Tensor], BT: int, ignore_index: int = -100,
+                device=None, out: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Kept rows of a batch (labels != ignore_index; all BT rows when labels is
+    None) as a device int64 scalar, counted by the CUDA library."""
+    dev = labels.device if labels is not None else torch.device(device or "cuda")
+    if labels is not None:
+        _check_dev("labels", labels, torch.int64, (BT,), dev)
+    count = torch.empty((), dtype=torch.int64, device=dev) if out is None else out
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    status = flkl_count_valid(_ptr(labels), BT, ignore_index, _ptr(count), st.cuda_stream)
+    if status != FLKL_OK:
+        raise FlklError(status, "flkl_count_valid")
+    return count
 
 
 class _FusedLinearCEFunction(torch.autograd.Function):

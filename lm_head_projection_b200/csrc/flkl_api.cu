@@ -504,7 +504,8 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
                                   int reduction, int compute_dW, int compute_db, int accum_fp32,
                                   float* loss, void* dX, void* dW, void* db, void* workspace,
                                   size_t workspace_bytes, void* stream, Recorder* rec,
-                                  const int64_t* target = nullptr) {
+                                  const int64_t* target = nullptr,
+                                  const int64_t* n_valid_total = nullptr) {
   // Cross-entropy mode (target set): the teacher is one-hot at target[row],
   // Q is not read and the target doubles as the row mask.
   if (target != nullptr) {
@@ -549,7 +550,7 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
     k_prepare<<<1, 1024, 0, st>>>(shift_labels, bt, static_cast<long long>(ignore_index),
                                   reduction, v, temperature, reinterpret_cast<DevCtl*>(ws),
                                   reinterpret_cast<int*>(ws + P.off_cnt),
-                                  static_cast<int>(P.n_counters));
+                                  static_cast<int>(P.n_counters), n_valid_total);
     FLKL_CUDA(cudaGetLastError());
   }
 
@@ -661,6 +662,49 @@ flkl_status flkl_ce_forward_backward(const void* X, const void* W, const void* b
                                temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
                                BT > 0 ? target : nullptr);
+}
+
+flkl_status flkl_count_valid(const int64_t* labels, int64_t BT, int64_t ignore_index,
+                             int64_t* count, void* stream) {
+  if (count == nullptr || BT < 0) return FLKL_ERR_INVALID_ARG;
+  if (BT >= (int64_t(1) << 31)) return FLKL_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(labels) & 7u) || (reinterpret_cast<uintptr_t>(count) & 7u))
+    return FLKL_ERR_UNSUPPORTED;
+  k_count_valid<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      BT > 0 ? labels : nullptr, static_cast<int>(BT), static_cast<long long>(ignore_index),
+      count);
+  return cudaGetLastError() == cudaSuccess ? FLKL_OK : FLKL_ERR_CUDA;
+}
+
+flkl_status flkl_forward_backward_dp(const void* X, const void* W, const void* b, const void* Q,
+                                     const int64_t* shift_labels, int64_t ignore_index,
+                                     int64_t BT, int64_t H, int64_t V, int dtype,
+                                     float temperature, float eps, int reduction, int compute_dW,
+                                     int compute_db, int accum_fp32, float* loss, void* dX,
+                                     void* dW, void* db, void* workspace, size_t workspace_bytes,
+                                     void* stream, const int64_t* n_valid_total) {
+  if (n_valid_total == nullptr || (reinterpret_cast<uintptr_t>(n_valid_total) & 7u))
+    return FLKL_ERR_INVALID_ARG;
+  return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                               temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
+                               nullptr, n_valid_total);
+}
+
+flkl_status flkl_ce_forward_backward_dp(const void* X, const void* W, const void* b,
+                                        const int64_t* target, int64_t ignore_index, int64_t BT,
+                                        int64_t H, int64_t V, int dtype, float temperature,
+                                        int reduction, int compute_dW, int compute_db,
+                                        int accum_fp32, float* loss, void* dX, void* dW, void* db,
+                                        void* workspace, size_t workspace_bytes, void* stream,
+                                        const int64_t* n_valid_total) {
+  if (BT > 0 && target == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (n_valid_total == nullptr || (reinterpret_cast<uintptr_t>(n_valid_total) & 7u))
+    return FLKL_ERR_INVALID_ARG;
+  return forward_backward_impl(X, W, b, nullptr, nullptr, ignore_index, BT, H, V, dtype,
+                               temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
+                               BT > 0 ? target : nullptr, n_valid_total);
 }
 
 flkl_status flkl_forward_backward_profiled(

@@ -319,17 +319,20 @@ __global__ void __launch_bounds__(kColsumThreads)
   void* out = blockIdx.y ? out1 : out0;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + lane;
+  // 16 loads in flight per thread, then added in order (a missing row adds 0)
+  constexpr int U = 16;
   float s = 0.f;
   if (c < H) {
-    int b = warp;
-    for (; b + 3 * NWc < nblocks; b += 4 * NWc) {
-      const float v0 = part[static_cast<size_t>(b) * H + c];
-      const float v1 = part[static_cast<size_t>(b + NWc) * H + c];
-      const float v2 = part[static_cast<size_t>(b + 2 * NWc) * H + c];
-      const float v3 = part[static_cast<size_t>(b + 3 * NWc) * H + c];
-      s = (((s + v0) + v1) + v2) + v3;
+    for (int b0 = warp; b0 < nblocks; b0 += U * NWc) {
+      float v[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int b = b0 + j * NWc;
+        v[j] = b < nblocks ? part[static_cast<size_t>(b) * H + c] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j) s += v[j];
     }
-    for (; b < nblocks; b += NWc) s += part[static_cast<size_t>(b) * H + c];
   }
   sl[warp][lane] = s;
   __syncthreads();

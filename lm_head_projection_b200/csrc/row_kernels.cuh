@@ -10,7 +10,7 @@ namespace flkl {
 // Device-side control block at the start of the workspace.
 struct DevCtl {
   int err;       // first device error code of the call (0 = none)
-  int n_valid;   // rows whose shift label differs from ignore_index
+  int n_valid;   // rows of this call whose shift label differs from ignore_index
   float D;       // reduction divisor
   float scale;   // 1 / (T * D), 0 when no row is kept
   float invD;    // 1 / D, 0 when no row is kept
@@ -19,11 +19,14 @@ struct DevCtl {
 // One block of 1024 threads.  Counts kept rows (a row is dropped when its
 // shift label equals ignore_index), derives the divisor of the reduction
 // (batchmean: N_valid, mean: N_valid * V, sum: 1), resets the error flag and
-// zeroes the tile counters of the call's persistent launches.
+// zeroes the tile counters of the call's persistent launches.  With
+// `n_total` (data-parallel use) the divisor counts *n_total kept rows, the
+// kept rows of every rank's batch, instead of this call's.
 __global__ void __launch_bounds__(1024) k_prepare(const int64_t* __restrict__ labels, int BT,
                                                   long long ignore_index, int reduction, int V,
                                                   float temperature, DevCtl* ctl,
-                                                  int* counters, int n_counters) {
+                                                  int* counters, int n_counters,
+                                                  const int64_t* __restrict__ n_total) {
   __shared__ int warp_cnt[32];
   for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
   int cnt = 0;
@@ -37,16 +40,38 @@ __global__ void __launch_bounds__(1024) k_prepare(const int64_t* __restrict__ la
   if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
   __syncthreads();
   if (threadIdx.x == 0) {
-    int n = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) n += warp_cnt[w];
+    int n_local = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) n_local += warp_cnt[w];
+    const long long n = n_total != nullptr ? *n_total : n_local;
     float D = 1.f;
     if (reduction == 0) D = static_cast<float>(n);
     else if (reduction == 1) D = static_cast<float>(n) * static_cast<float>(V);
     ctl->err = 0;
-    ctl->n_valid = n;
+    ctl->n_valid = n_local;
     ctl->D = D;
     ctl->scale = n > 0 ? 1.f / (temperature * D) : 0.f;
     ctl->invD = n > 0 ? 1.f / D : 0.f;
+  }
+}
+
+// Kept rows of one batch (labels NULL: all BT rows) into *count (int64).
+__global__ void __launch_bounds__(1024) k_count_valid(const int64_t* __restrict__ labels, int BT,
+                                                      long long ignore_index, int64_t* count) {
+  __shared__ int warp_cnt[32];
+  int cnt = 0;
+  if (labels == nullptr) {
+    cnt = (threadIdx.x == 0) ? BT : 0;
+  } else {
+    for (int i = threadIdx.x; i < BT; i += blockDim.x) cnt += (labels[i] != ignore_index) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) warp_cnt[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long n = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) n += warp_cnt[w];
+    *count = n;
   }
 }
 

@@ -1,0 +1,113 @@
+"""Data-parallel form of the fused loss on one GPU: the kept-row count of the
+CUDA library, the divisor taken from a whole-batch count (rows split in two
+calls add up to the whole batch), and DataParallelFusedLinearLoss over a
+one-rank NCCL group giving the direct call's bytes.
+"""
+
+from __future__ import annotations
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+from lm_head_projection_b200.workloads import make_inputs, small_case
+from parity_utils import TOL, assert_close, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _call(pkg, g, rows=None, n_total=None):
+    sl = (lambda t: t) if rows is None else (lambda t: None if t is None else t[rows])
+    common = dict(compute_dW=True, compute_db=g["compute_db"], accum_fp32=True,
+                  n_valid_total=n_total, check_status=True)
+    if g.get("target") is not None:
+        return pkg.cross_entropy_forward_backward(sl(g["X"]).contiguous(), g["W"], g["b"],
+                                                  sl(g["target"]).contiguous(),
+                                                  g["ignore_index"], g["temperature"],
+                                                  g["reduction"], **common)
+    lab = g["shift_labels"]
+    return pkg.forward_backward(sl(g["X"]).contiguous(), g["W"], g["b"],
+                                sl(g["Q"]).contiguous(),
+                                None if lab is None else sl(lab).contiguous(), g["ignore_index"],
+                                g["temperature"], g["eps"], g["reduction"], **common)
+
+
+def test_count_valid():
+    import lm_head_projection_b200 as pkg
+
+    lab = torch.tensor([3, -100, 7, -100, -100, 0], dtype=torch.int64, device="cuda")
+    assert int(pkg.count_valid(lab, 6)) == 3
+    assert int(pkg.count_valid(None, 11, device="cuda")) == 11
+    assert int(pkg.count_valid(lab[:0], 0)) == 0
+    big = torch.full((100_000,), -100, dtype=torch.int64, device="cuda")
+    big[::7] = 1
+    assert int(pkg.count_valid(big, big.numel())) == int((big != -100).sum())
+
+
+@pytest.mark.parametrize("dtype,reduction,ce", [("fp32", "batchmean", False),
+                                               ("bf16", "mean", False),
+                                               ("bf16", "sum", False),
+                                               ("bf16", "batchmean", True),
+                                               ("fp32", "mean", True)])
+def test_split_rows_with_whole_batch_count_add_up(dtype, reduction, ce):
+    import lm_head_projection_b200 as pkg
+
+    w = small_case(dtype=dtype, BT=203, H=128 if dtype == "bf16" else 64, V=1000,
+                   bias=True, reduction=reduction, ignore_frac=0.2, temperature=1.5, ce=ce,
+                   seed=11)
+    inp = make_inputs(w)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    whole = _call(pkg, g)
+    mask = g["target"] if ce else g["shift_labels"]
+    n_total = pkg.count_valid(mask, w.BT)
+    halves = [torch.arange(0, 120, device="cuda"), torch.arange(120, w.BT, device="cuda")]
+    parts = [_call(pkg, g, rows, n_total) for rows in halves]
+    torch.cuda.synchronize()
+    got = {"loss": parts[0]["loss"] + parts[1]["loss"],
+           "dX": torch.cat([parts[0]["dX"], parts[1]["dX"]]),
+           "dW": parts[0]["dW"] + parts[1]["dW"],
+           "db": parts[0]["db"] + parts[1]["db"]}
+    ref = run_oracle(inp, compute_dW=True, compute_db=True)
+    assert_close(dtype, got, ref)
+    # the split halves and the whole-batch call agree within the same bound
+    assert_close(dtype, got, {k: (float(v.double().cpu()) if k == "loss" else
+                                  v.double().cpu().numpy()) for k, v in whole.items()
+                              if k in ("loss", "dX", "dW", "db")})
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("kind", ["kl", "ce"])
+def test_one_rank_nccl_group_gives_the_direct_call(kind):
+    import torch.distributed as dist
+
+    import lm_head_projection_b200 as pkg
+    from lm_head_projection_b200.dp import DataParallelFusedLinearLoss
+
+    w = small_case(dtype="bf16", BT=300, H=256, V=2000, bias=True, ignore_frac=0.1,
+                   ce=(kind == "ce"), seed=5)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v)
+         for k, v in make_inputs(w).items()}
+    direct = _call(pkg, g)
+    torch.cuda.synchronize()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda:0"))
+    try:
+        loss = DataParallelFusedLinearLoss(kind, temperature=w.temperature, eps=w.eps)
+        teacher = g["target"] if kind == "ce" else g["Q"]
+        r = loss.step(g["X"], g["W"], g["b"], teacher, g["shift_labels"], compute_dW=True,
+                      compute_db=True)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    for k in ("loss", "dX", "dW", "db"):
+        assert torch.equal(r[k], direct[k]), k
