@@ -148,6 +148,34 @@ FLKL_API flkl_status flkl_ce_forward_backward(const void* X, const void* W, cons
                                               void* dX, void* dW, void* db, void* workspace,
                                               size_t workspace_bytes, void* stream);
 
+/* Selective log-probability (the GRPO frozen-head page, Summary: the chunked
+ * per-token log-probability of the policy head, whose weight and bias
+ * gradients are computed only when they are asked for).  Two calls on the
+ * same workspace:
+ *
+ * flkl_selective_logprob_forward: logp[r] = z_{r,t}/T - logsumexp_v(z_{r,v}/T)
+ *   with z = X W^T (+ b) and t = target[r]; 0 on rows whose target is
+ *   ignore_index or outside [0, V).  logp: device fp32 [BT].  compute_dW /
+ *   compute_db size the workspace (flkl_workspace_size with the same flags)
+ *   for the backward call; nothing else is written.  The workspace keeps the
+ *   row statistics for the backward call: do not use it for another call in
+ *   between.
+ * flkl_selective_logprob_backward: for upstream gradients dlogp [BT] (device
+ *   fp32), dz_r = dlogp[r] (onehot(t) - softmax(z_r/T)) / T, and dX = dz W,
+ *   dW = dz^T X (compute_dW), db = column sums of dz (compute_db), written as
+ *   in flkl_forward_backward.  X, W, b, target, ignore_index, sizes, dtype,
+ *   temperature and the flags must be those of the forward call.
+ * Errors, alignment and asynchrony as flkl_forward_backward. */
+FLKL_API flkl_status flkl_selective_logprob_forward(
+    const void* X, const void* W, const void* b, const int64_t* target, int64_t ignore_index,
+    int64_t BT, int64_t H, int64_t V, int dtype, float temperature, int compute_dW,
+    int compute_db, float* logp, void* workspace, size_t workspace_bytes, void* stream);
+FLKL_API flkl_status flkl_selective_logprob_backward(
+    const void* X, const void* W, const void* b, const int64_t* target, int64_t ignore_index,
+    int64_t BT, int64_t H, int64_t V, int dtype, float temperature, const float* dlogp,
+    int compute_dW, int compute_db, int accum_fp32, void* dX, void* dW, void* db,
+    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Data-parallel use: the batch is split by rows over ranks that share the
  * head W, b (the row sharding of the scope table's multi-GPU row).  Each rank
  * calls flkl_count_valid on its labels (or targets), all-reduces the int64

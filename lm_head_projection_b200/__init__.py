@@ -23,7 +23,8 @@ __all__ = [
     "flkl_ce_forward_backward", "cross_entropy_forward_backward", "FusedLinearCrossEntropyLoss",
     "flkl_norm_workspace_size", "flkl_rms_norm_backward", "flkl_layer_norm_backward",
     "flkl_norm_device_status", "flkl_count_valid", "flkl_forward_backward_dp",
-    "flkl_ce_forward_backward_dp", "count_valid",
+    "flkl_ce_forward_backward_dp", "count_valid", "flkl_selective_logprob_forward",
+    "flkl_selective_logprob_backward", "selective_logprob", "SelectiveLogProb",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +87,16 @@ def _lib():
         lib.flkl_ce_forward_backward_dp.restype = c.c_int
         lib.flkl_ce_forward_backward_dp.argtypes = list(
             lib.flkl_ce_forward_backward.argtypes) + [c.c_void_p]
+        lib.flkl_selective_logprob_forward.restype = c.c_int
+        lib.flkl_selective_logprob_forward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int64,
+            c.c_int64, c.c_int, c.c_float, c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_size_t,
+            c.c_void_p]
+        lib.flkl_selective_logprob_backward.restype = c.c_int
+        lib.flkl_selective_logprob_backward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int64,
+            c.c_int64, c.c_int, c.c_float, c.c_void_p, c.c_int, c.c_int, c.c_int, c.c_void_p,
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
         lib.flkl_count_valid.restype = c.c_int
         lib.flkl_count_valid.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p]
         lib.flkl_forward_backward_noalloc.restype = c.c_int
@@ -180,6 +191,26 @@ def flkl_ce_forward_backward_dp(X, W, b, target, ignore_index, BT, H, V, dtype, 
         float(temperature), int(reduction), int(bool(compute_dW)), int(bool(compute_db)),
         int(bool(accum_fp32)), loss, dX, dW, db, workspace, int(workspace_bytes), stream,
         n_valid_total)
+
+
+def flkl_selective_logprob_forward(X, W, b, target, ignore_index, BT, H, V, dtype, temperature,
+                                   compute_dW, compute_db, logp, workspace, workspace_bytes,
+                                   stream) -> int:
+    """Per-row target log-probabilities (raw pointers); returns the status."""
+    return _lib().flkl_selective_logprob_forward(
+        X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), int(bool(compute_dW)), int(bool(compute_db)), logp, workspace,
+        int(workspace_bytes), stream)
+
+
+def flkl_selective_logprob_backward(X, W, b, target, ignore_index, BT, H, V, dtype, temperature,
+                                    dlogp, compute_dW, compute_db, accum_fp32, dX, dW, db,
+                                    workspace, workspace_bytes, stream) -> int:
+    """Gradients for upstream per-row gradients ``dlogp`` (raw pointers)."""
+    return _lib().flkl_selective_logprob_backward(
+        X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
+        float(temperature), dlogp, int(bool(compute_dW)), int(bool(compute_db)),
+        int(bool(accum_fp32)), dX, dW, db, workspace, int(workspace_bytes), stream)
 
 
 def flkl_norm_workspace_size(rows, H, compute_dW, compute_db) -> int:
@@ -484,6 +515,99 @@ def count_valid(labels: Optional[torch.Tensor], BT: int, ignore_index: int = -10
     if status != FLKL_OK:
         raise FlklError(status, "flkl_count_valid")
     return count
+
+
+class _SelectiveLogProbFunction(torch.autograd.Function):
+    """Per-row target log-probabilities with a true backward: the forward
+    keeps the row statistics in its workspace, the backward runs pass 2 and
+    the dX / dW / db GEMMs for the incoming gradients, computing dW and db
+    only when autograd asks for them."""
+
+    @staticmethod
+    def forward(ctx, X, W, b, target, ignore_index, temperature, accum_fp32):
+        X, W = X.contiguous(), W.contiguous()
+        b = None if b is None else b.contiguous()
+        target = target.contiguous()
+        dev, dt = X.device, X.dtype
+        if dt not in DTYPES:
+            raise ValueError(f"dtype {dt} not supported (float32 or bfloat16)")
+        BT, H = X.shape
+        V = W.shape[0]
+        _check_dev("W", W, dt, (V, H), dev)
+        _check_dev("target", target, torch.int64, (BT,), dev)
+        if b is not None:
+            _check_dev("b", b, dt, (V,), dev)
+        cw = bool(ctx.needs_input_grad[1])
+        cb = bool(b is not None and ctx.needs_input_grad[2])
+        need = flkl_workspace_size(BT, H, V, DTYPES[dt], cw, cb)
+        if need == 0:
+            raise FlklError(1, "flkl_workspace_size")
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        logp = torch.empty((BT,), dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream(dev)
+        s = flkl_selective_logprob_forward(_ptr(X), _ptr(W), _ptr(b), _ptr(target),
+                                           ignore_index, BT, H, V, DTYPES[dt], temperature, cw,
+                                           cb, _ptr(logp), _ptr(ws), ws.numel(), st.cuda_stream)
+        if s != FLKL_OK:
+            raise FlklError(s, "flkl_selective_logprob_forward")
+        ctx.save_for_backward(X, W, b, target)
+        ctx.ws, ctx.cw, ctx.cb = ws, cw, cb
+        ctx.opts = (ignore_index, temperature, accum_fp32)
+        return logp
+
+    @staticmethod
+    def backward(ctx, dlogp):
+        X, W, b, target = ctx.saved_tensors
+        ignore_index, temperature, accum_fp32 = ctx.opts
+        dev, dt = X.device, X.dtype
+        BT, H = X.shape
+        V = W.shape[0]
+        dlogp = dlogp.contiguous().to(torch.float32)
+        pdt = torch.float32 if (accum_fp32 or dt == torch.float32) else dt
+        dX = torch.empty_like(X)
+        dW = torch.empty((V, H), dtype=pdt, device=dev) if ctx.cw else None
+        db = torch.empty((V,), dtype=pdt, device=dev) if ctx.cb else None
+        st = torch.cuda.current_stream(dev)
+        s = flkl_selective_logprob_backward(
+            _ptr(X), _ptr(W), _ptr(b), _ptr(target), ignore_index, BT, H, V, DTYPES[dt],
+            temperature, _ptr(dlogp), ctx.cw, ctx.cb, accum_fp32, _ptr(dX), _ptr(dW), _ptr(db),
+            _ptr(ctx.ws), ctx.ws.numel(), st.cuda_stream)
+        if s != FLKL_OK:
+            raise FlklError(s, "flkl_selective_logprob_backward")
+        ctx.ws = None
+        if dW is not None:
+            dW = dW.to(W.dtype)
+        if db is not None:
+            db = db.to(W.dtype)
+        return dX, dW, db, None, None, None, None
+
+
+def selective_logprob(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor],
+                      target: torch.Tensor, ignore_index: int = -100,
+                      temperature: float = 1.0, accum_fp32: bool = True) -> torch.Tensor:
+    """Per-row log-probability of ``target`` under softmax((X Wᵀ + b)/T), as
+    an autograd function (any loss of the per-token log-probabilities can
+    follow, e.g. a policy-gradient objective); rows whose target is
+    ``ignore_index`` or outside [0, V) give 0 and no gradient.  dW / db are
+    computed only when W / b require grad."""
+    return _SelectiveLogProbFunction.apply(X, W, b, target, ignore_index, temperature,
+                                           accum_fp32)
+
+
+class SelectiveLogProb(torch.nn.Module):
+    """Module form of :func:`selective_logprob`:
+    ``forward(lin_weight, _input, target, bias=None) -> logp [BT]``."""
+
+    def __init__(self, ignore_index: int = -100, temperature: float = 1.0,
+                 accum_dtype: Optional[torch.dtype] = torch.float32):
+        super().__init__()
+        self.ignore_index = ignore_index
+        self.temperature = temperature
+        self.accum_fp32 = accum_dtype == torch.float32
+
+    def forward(self, lin_weight, _input, target, bias=None):
+        return selective_logprob(_input, lin_weight, bias, target, self.ignore_index,
+                                 self.temperature, self.accum_fp32)
 
 
 class _FusedLinearCEFunction(torch.autograd.Function):

@@ -263,12 +263,55 @@ struct Rec {
     if ((x) != cudaSuccess) return FLKL_ERR_CUDA;  \
   } while (0)
 
+// Which parts of the path a call runs.  The whole call (forward_backward)
+// runs both; the selective log-probability entries run the forward part
+// (statistics, per-row log-probabilities into `logp`) and, in a later call on
+// the same workspace, the backward part with upstream gradients `dlogp`.
+struct Phases {
+  bool forward = true;
+  bool backward = true;
+  float* logp = nullptr;         // forward: per-row output instead of the loss
+  const float* dlogp = nullptr;  // backward: per-row upstream gradients
+};
+
+// Merge of the statistics into row values, then the reduced loss and / or the
+// per-row log-probabilities.
+cudaError_t finish_rows(const Plan& P, const float* stats, int BT, const int64_t* labels,
+                        long long ignore_index, float T, DevCtl* ctl, float* lse2, float* coefS,
+                        float* coefQ, float* rowloss, float* loss, float* logp, cudaStream_t st,
+                        Recorder* rec) {
+  {
+    Rec r_(rec, 2);
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
+        stats, static_cast<int>(P.n_stat), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
+        coefQ, rowloss);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  Rec r_(rec, 3);
+  if (loss != nullptr) k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
+  if (logp != nullptr)
+    k_neg_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(rowloss, BT, logp);
+  return cudaGetLastError();
+}
+
+// Backward with upstream per-row gradients: replaces the row coefficients.
+cudaError_t upstream_coefs(const float* dlogp, const int64_t* target, int BT,
+                           long long ignore_index, int V, float T, float* coefS, float* coefQ,
+                           cudaStream_t st, Recorder* rec) {
+  if (dlogp == nullptr) return cudaSuccess;
+  Rec r_(rec, 2);
+  k_coef_from_dlogp<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
+      dlogp, target, BT, ignore_index, V, 1.f / T, coefS, coefQ);
+  return cudaGetLastError();
+}
+
 flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W,
                    const __nv_bfloat16* b, const __nv_bfloat16* Q, const int64_t* labels,
                    long long ignore_index, int BT, int H, int V, float T, float eps,
                    int compute_dW, int compute_db, int accum_fp32, float* loss,
                    __nv_bfloat16* dX, void* dW, void* db, uint8_t* ws, cudaStream_t st,
-                   Recorder* rec, const int64_t* target) {
+                   Recorder* rec, const int64_t* target, const Phases& ph) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   int* counters = reinterpret_cast<int*>(ws + P.off_cnt);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
@@ -311,26 +354,20 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     return add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, c0, 0);
   };
 
-  // pass 1: statistics over all V
-  {
-    TcLaunch L = new_launch(0);
-    TcMaps maps{};
-    add_problem(L, maps, KIND_STATS, BT, V, H, 1, mX_k, mW_k);
-    Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
-    FLKL_CUDA(launch_group(maps, L, st));
+  if (ph.forward) {
+    // pass 1: statistics over all V
+    {
+      TcLaunch L = new_launch(0);
+      TcMaps maps{};
+      add_problem(L, maps, KIND_STATS, BT, V, H, 1, mX_k, mW_k);
+      Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
+      FLKL_CUDA(launch_group(maps, L, st));
+    }
+    FLKL_CUDA(finish_rows(P, stats, BT, labels, ignore_index, T, ctl, lse2, coefS, coefQ,
+                          rowloss, loss, ph.logp, st, rec));
   }
-  {
-    Rec r_(rec, 2);
-    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
-        stats, static_cast<int>(P.n_stat), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
-        coefQ, rowloss);
-    FLKL_CUDA(cudaGetLastError());
-  }
-  {
-    Rec r_(rec, 3);
-    k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
-    FLKL_CUDA(cudaGetLastError());
-  }
+  if (!ph.backward) return FLKL_OK;
+  FLKL_CUDA(upstream_coefs(ph.dlogp, target, BT, ignore_index, V, T, coefS, coefQ, st, rec));
   // pass 2 of chunk 0 alone
   {
     TcLaunch L = new_launch(1);
@@ -376,7 +413,7 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
                     const int64_t* labels, long long ignore_index, int BT, int H, int V, float T,
                     float eps, int compute_dW, int compute_db, float* loss, float* dX, float* dW,
                     float* db, uint8_t* ws, cudaStream_t st, Recorder* rec,
-                    const int64_t* target) {
+                    const int64_t* target, const Phases& ph) {
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
   float* rows = reinterpret_cast<float*>(ws + P.off_rows);
@@ -390,24 +427,19 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
   const float t_scale = 1.4426950408889634f / T;
   const unsigned mt = static_cast<unsigned>(P.m_tiles);
 
-  {
-  Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
-  k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
-      X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT, target);
-  FLKL_CUDA(cudaGetLastError());
+  if (ph.forward) {
+    {
+      Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
+      k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
+          X, W, b, Q, BT, H, V, t_scale, eps, stats, static_cast<long long>(P.n_tiles) * BT,
+          target);
+      FLKL_CUDA(cudaGetLastError());
+    }
+    FLKL_CUDA(finish_rows(P, stats, BT, labels, ignore_index, T, ctl, lse2, coefS, coefQ,
+                          rowloss, loss, ph.logp, st, rec));
   }
-  {
-    Rec r_(rec, 2);
-    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
-        stats, static_cast<int>(P.n_stat), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
-        coefQ, rowloss);
-    FLKL_CUDA(cudaGetLastError());
-  }
-  {
-    Rec r_(rec, 3);
-    k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
-    FLKL_CUDA(cudaGetLastError());
-  }
+  if (!ph.backward) return FLKL_OK;
+  FLKL_CUDA(upstream_coefs(ph.dlogp, target, BT, ignore_index, V, T, coefS, coefQ, st, rec));
 
   const int ldg = static_cast<int>(P.Vc);
   for (long long c = 0; c < P.nchunks; ++c) {
@@ -505,7 +537,8 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
                                   float* loss, void* dX, void* dW, void* db, void* workspace,
                                   size_t workspace_bytes, void* stream, Recorder* rec,
                                   const int64_t* target = nullptr,
-                                  const int64_t* n_valid_total = nullptr) {
+                                  const int64_t* n_valid_total = nullptr,
+                                  const Phases& ph = Phases{}) {
   // Cross-entropy mode (target set): the teacher is one-hot at target[row],
   // Q is not read and the target doubles as the row mask.
   if (target != nullptr) {
@@ -525,11 +558,16 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
   const int vec = dtype == FLKL_DTYPE_BF16 ? 8 : 4;
   if (H % vec != 0 || V % vec != 0) return FLKL_ERR_UNSUPPORTED;
   // ---- pointers
-  if (W == nullptr || loss == nullptr) return FLKL_ERR_INVALID_ARG;
-  if (BT > 0 && (X == nullptr || (Q == nullptr && target == nullptr) || dX == nullptr))
-    return FLKL_ERR_INVALID_ARG;
-  if ((compute_dW != 0) != (dW != nullptr)) return FLKL_ERR_INVALID_ARG;
-  if ((compute_db != 0) != (db != nullptr)) return FLKL_ERR_INVALID_ARG;
+  if (W == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (ph.forward && loss == nullptr && ph.logp == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (BT > 0 && (X == nullptr || (Q == nullptr && target == nullptr))) return FLKL_ERR_INVALID_ARG;
+  if (ph.backward) {
+    // outputs of the backward part (a forward-only call writes none of them;
+    // its flags only size the workspace the backward call will use)
+    if (BT > 0 && dX == nullptr) return FLKL_ERR_INVALID_ARG;
+    if ((compute_dW != 0) != (dW != nullptr)) return FLKL_ERR_INVALID_ARG;
+    if ((compute_db != 0) != (db != nullptr)) return FLKL_ERR_INVALID_ARG;
+  }
   if (compute_db && b == nullptr) return FLKL_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(b) || !aligned16(Q) || !aligned16(dX) ||
       !aligned16(dW) || !aligned16(db) || (reinterpret_cast<uintptr_t>(shift_labels) & 7u) ||
@@ -557,8 +595,9 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
   if (BT == 0) {
     // No rows: loss 0, and zero parameter gradients when asked for.
     Rec r_(rec, 8);
-    k_zero<<<1, 32, 0, st>>>(loss, sizeof(float));
+    if (loss != nullptr) k_zero<<<1, 32, 0, st>>>(loss, sizeof(float));
     FLKL_CUDA(cudaGetLastError());
+    if (!ph.backward) return FLKL_OK;
     const size_t pe = (dtype == FLKL_DTYPE_F32 || accum_fp32) ? 4 : 2;
     if (compute_dW) {
       const size_t bytes = size_t(V) * H * pe;
@@ -577,13 +616,14 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
     return run_tc(P, static_cast<const __nv_bfloat16*>(X), static_cast<const __nv_bfloat16*>(W),
                   static_cast<const __nv_bfloat16*>(b), static_cast<const __nv_bfloat16*>(Q),
                   shift_labels, ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db,
-                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st, rec, target);
+                  accum_fp32, loss, static_cast<__nv_bfloat16*>(dX), dW, db, ws, st, rec, target,
+                  ph);
   }
   return run_f32(P, static_cast<const float*>(X), static_cast<const float*>(W),
                  static_cast<const float*>(b), static_cast<const float*>(Q), shift_labels,
                  ignore_index, bt, h, v, temperature, eps, compute_dW, compute_db, loss,
                  static_cast<float*>(dX), static_cast<float*>(dW), static_cast<float*>(db), ws,
-                 st, rec, target);
+                 st, rec, target, ph);
 }
 
 // Fixed scratch of flkl_forward_backward_noalloc (see flkl.h): part of the
@@ -705,6 +745,41 @@ flkl_status flkl_ce_forward_backward_dp(const void* X, const void* W, const void
                                temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
                                BT > 0 ? target : nullptr, n_valid_total);
+}
+
+flkl_status flkl_selective_logprob_forward(const void* X, const void* W, const void* b,
+                                           const int64_t* target, int64_t ignore_index,
+                                           int64_t BT, int64_t H, int64_t V, int dtype,
+                                           float temperature, int compute_dW, int compute_db,
+                                           float* logp, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+  if (BT > 0 && (target == nullptr || logp == nullptr)) return FLKL_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(logp) & 3u) return FLKL_ERR_UNSUPPORTED;
+  Phases ph;
+  ph.backward = false;
+  ph.logp = logp;
+  return forward_backward_impl(X, W, b, nullptr, nullptr, ignore_index, BT, H, V, dtype,
+                               temperature, 0.f, FLKL_REDUCTION_SUM, compute_dW, compute_db, 1,
+                               nullptr, nullptr, nullptr, nullptr, workspace, workspace_bytes,
+                               stream, nullptr, BT > 0 ? target : nullptr, nullptr, ph);
+}
+
+flkl_status flkl_selective_logprob_backward(const void* X, const void* W, const void* b,
+                                            const int64_t* target, int64_t ignore_index,
+                                            int64_t BT, int64_t H, int64_t V, int dtype,
+                                            float temperature, const float* dlogp,
+                                            int compute_dW, int compute_db, int accum_fp32,
+                                            void* dX, void* dW, void* db, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+  if (BT > 0 && (target == nullptr || dlogp == nullptr)) return FLKL_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(dlogp) & 3u) return FLKL_ERR_UNSUPPORTED;
+  Phases ph;
+  ph.forward = false;
+  ph.dlogp = dlogp;
+  return forward_backward_impl(X, W, b, nullptr, nullptr, ignore_index, BT, H, V, dtype,
+                               temperature, 0.f, FLKL_REDUCTION_SUM, compute_dW, compute_db,
+                               accum_fp32, nullptr, dX, dW, db, workspace, workspace_bytes,
+                               stream, nullptr, BT > 0 ? target : nullptr, nullptr, ph);
 }
 
 flkl_status flkl_forward_backward_profiled(

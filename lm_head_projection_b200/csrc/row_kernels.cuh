@@ -75,6 +75,31 @@ __global__ void __launch_bounds__(1024) k_count_valid(const int64_t* __restrict_
   }
 }
 
+// Selective log-probability (cross-entropy mode): logp[r] = -rowloss[r], the
+// log-probability of row r's target (0 on dropped rows and on targets
+// outside [0, V)).
+__global__ void k_neg_rows(const float* __restrict__ rowloss, int BT, float* __restrict__ out) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r < BT) out[r] = -rowloss[r];
+}
+
+// Row coefficients of the selective log-probability backward: for an
+// upstream gradient dlogp[r], dz_r = dlogp[r] (onehot(target_r) - p_r) / T,
+// which is the pass-2 form G = coefS p - coefQ onehot with coefS = coefQ =
+// -dlogp[r] / T; 0 on dropped rows and on targets outside [0, V).
+__global__ void k_coef_from_dlogp(const float* __restrict__ dlogp,
+                                  const int64_t* __restrict__ target, int BT,
+                                  long long ignore_index, int V, float invT,
+                                  float* __restrict__ coefS, float* __restrict__ coefQ) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= BT) return;
+  const long long y = target[r];
+  const bool keep = y != ignore_index && y >= 0 && y < V;
+  const float c = keep ? -dlogp[r] * invT : 0.f;
+  coefS[r] = c;
+  coefQ[r] = c;
+}
+
 // Merge of the per-group statistics (m, s, A, B2, S) of each row, in group
 // order, into lse2 = log2 sum 2^t and the row loss
 //   l_r = ln2 * B2 - A / T + ln2 * lse2 * S

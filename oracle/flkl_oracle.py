@@ -284,3 +284,80 @@ def ce_forward_backward(X, W, b, target, ignore_index=-100, temperature=1.0,
             db += G.sum(axis=0)
     loss = 0.0 if n_valid == 0 else float(row_loss.sum() / D)
     return dict(loss=loss, dX=dX, dW=dW, db=db, row_loss=row_loss, n_valid=n_valid, D=D)
+
+
+def selective_logprob(X, W, b, target, ignore_index=-100, temperature=1.0, row_block=256):
+    """Per-row log-probability of the target, fp64 (the chunked selective
+    log-probability of the GRPO frozen-head page, *Summary*):
+
+        logp_r = u_{r, y_r} - lse(u_r),   u = (X W^T + b) / T,
+
+    0 on rows whose target is ignore_index or outside [0, V)."""
+    BT = np.shape(X)[0]
+    V = np.shape(W)[0]
+    T = float(temperature)
+    tgt = np.asarray(target).astype(np.int64)
+    W64 = _as64(W)
+    b64 = _as64(b)
+    out = np.zeros(BT)
+    for r0 in range(0, BT, row_block):
+        r1 = min(BT, r0 + row_block)
+        z = _as64(X[r0:r1]) @ W64.T
+        if b64 is not None:
+            z += b64
+        logp, _ = log_softmax_rows(z / T)
+        y = tgt[r0:r1]
+        inside = (y != np.int64(ignore_index)) & (y >= 0) & (y < V)
+        rows = np.arange(r1 - r0)
+        out[r0:r1] = np.where(inside, logp[rows, np.clip(y, 0, V - 1)], 0.0)
+    return out
+
+
+def selective_logprob_backward(X, W, b, target, dlogp, ignore_index=-100, temperature=1.0,
+                               compute_dW=True, compute_db=False, dX_rows=None, dW_rows=None,
+                               row_block=256):
+    """Gradients of sum_r dlogp_r * logp_r (logp of :func:`selective_logprob`)
+    for given upstream gradients dlogp, fp64:
+
+        d / d z_rv = dlogp_r ([v == y_r] - p_rv) / T,   p_r = softmax(u_r),
+
+    zero on the rows whose logp is 0 by definition; dX = dz W, dW = dz^T X,
+    db = sum over rows of dz."""
+    if compute_db and b is None:
+        raise OracleError("compute_db needs a bias")
+    BT, H = np.shape(X)
+    V = np.shape(W)[0]
+    T = float(temperature)
+    tgt = np.asarray(target).astype(np.int64)
+    g = np.asarray(dlogp, dtype=np.float64)
+    W64 = _as64(W)
+    b64 = _as64(b)
+    dx_sel = np.arange(BT) if dX_rows is None else np.asarray(dX_rows, dtype=np.int64)
+    dw_sel = None if not compute_dW else (np.arange(V) if dW_rows is None
+                                          else np.asarray(dW_rows, dtype=np.int64))
+    dX = np.zeros((len(dx_sel), H))
+    dW = None if dw_sel is None else np.zeros((len(dw_sel), H))
+    db = np.zeros(V) if compute_db else None
+    dx_pos = {int(r): i for i, r in enumerate(dx_sel)}
+    for r0 in range(0, BT, row_block):
+        r1 = min(BT, r0 + row_block)
+        Xc = _as64(X[r0:r1])
+        z = Xc @ W64.T
+        if b64 is not None:
+            z += b64
+        logp, _ = log_softmax_rows(z / T)
+        y = tgt[r0:r1]
+        inside = (y != np.int64(ignore_index)) & (y >= 0) & (y < V)
+        rows = np.arange(r1 - r0)
+        G = -np.exp(logp)
+        G[rows[inside], np.clip(y, 0, V - 1)[inside]] += 1.0
+        G *= (g[r0:r1] / T)[:, None]
+        G[~inside] = 0.0
+        here = [i for i in range(r0, r1) if i in dx_pos]
+        if here:
+            dX[[dx_pos[i] for i in here]] = G[np.asarray(here) - r0] @ W64
+        if dW is not None:
+            dW += G[:, dw_sel].T @ Xc
+        if db is not None:
+            db += G.sum(axis=0)
+    return dict(dX=dX, dW=dW, db=db)

@@ -195,3 +195,26 @@ def test_norm_host_rejects_bad_arguments(layer, kw, expect):
 def test_layer_norm_bias_flag_needs_pointer():
     assert norm_call(True, compute_db=1) == INVALID            # db missing
     assert norm_call(True, compute_db=0, db=P) == INVALID      # db not asked for
+
+
+@no_gpu
+def test_selective_logprob_entries_check_their_arguments():
+    fwd = lambda **kw: pkg.flkl_selective_logprob_forward(**{**dict(
+        X=P, W=P, b=None, target=P, ignore_index=-100, BT=64, H=64, V=64, dtype=1,
+        temperature=1.0, compute_dW=1, compute_db=0, logp=P, workspace=P,
+        workspace_bytes=1 << 30, stream=None), **kw})
+    bwd = lambda **kw: pkg.flkl_selective_logprob_backward(**{**dict(
+        X=P, W=P, b=None, target=P, ignore_index=-100, BT=64, H=64, V=64, dtype=1,
+        temperature=1.0, dlogp=P, compute_dW=1, compute_db=0, accum_fp32=1, dX=P, dW=P,
+        db=None, workspace=P, workspace_bytes=1 << 30, stream=None), **kw})
+    assert fwd(target=None) == INVALID
+    assert fwd(logp=None) == INVALID
+    assert fwd(logp=P + 2) == UNSUPPORTED
+    assert fwd(temperature=0.0) == INVALID
+    assert fwd(workspace_bytes=16) == WORKSPACE
+    assert fwd(compute_db=1) == INVALID          # db needs a bias
+    assert bwd(dlogp=None) == INVALID
+    assert bwd(target=None) == INVALID
+    assert bwd(dX=None) == INVALID
+    assert bwd(dW=None) == INVALID               # compute_dW without dW
+    assert bwd(H=60) == UNSUPPORTED
