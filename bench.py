@@ -103,9 +103,11 @@ def parse():
     ap.add_argument("--cpu-sample-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", default="loss", choices=["loss", "rms_norm", "layer_norm"],
+    ap.add_argument("--op", default="loss",
+                    choices=["loss", "rms_norm", "layer_norm", "logprob"],
                     help="loss: the fused linear KL / CE loss (default); rms_norm / "
-                         "layer_norm: the norm backward with frozen-parameter flags")
+                         "layer_norm: the norm backward with frozen-parameter flags; logprob: "
+                         "selective log-probability forward + backward on a CE workload")
     ap.add_argument("--norm-shape", default="8192x8192", help="ROWSxH for --op *_norm")
     ap.add_argument("--norm-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--frozen", action="store_true", help="norm weight (and bias) frozen")
@@ -608,9 +610,100 @@ def run_norm(args):
     print(json.dumps(line), flush=True)
 
 
+def run_logprob(args):
+    """Selective log-probability on one GPU: one step = the forward call
+    (per-row target log-probabilities) and the backward call for upstream
+    gradients (dX, dW), on the cross-entropy workload's inputs; CUDA events
+    around exactly K steps."""
+    import numpy as np
+
+    import lm_head_projection_b200 as pkg
+    from lm_head_projection_b200.workloads import CE_WORKLOADS
+
+    name = args.workload if args.workload in CE_WORKLOADS else "ce_bf16_bt1024_h4096_v128256"
+    w = CE_WORKLOADS[name]
+    dev = torch.device("cuda", 0)
+    inp = make_inputs(w, device=dev)
+    X, W, b, tgt = inp["X"], inp["W"], inp["b"], inp["target"]
+    dt = pkg.DTYPES[X.dtype]
+    cw, cb = bool(w.compute_dW), bool(inp["compute_db"])
+    ws = torch.empty(pkg.flkl_workspace_size(w.BT, w.H, w.V, dt, cw, cb), dtype=torch.uint8,
+                     device=dev)
+    logp = torch.empty(w.BT, dtype=torch.float32, device=dev)
+    dlogp = torch.randn(w.BT, generator=torch.Generator(device=dev).manual_seed(1),
+                        device=dev, dtype=torch.float32)
+    dX = torch.empty_like(X)
+    dW = torch.empty((w.V, w.H), dtype=torch.float32, device=dev) if cw else None
+    db = torch.empty((w.V,), dtype=torch.float32, device=dev) if cb else None
+    p = lambda t: None if t is None else t.data_ptr()
+    stream = torch.cuda.current_stream(dev)
+    fa = (p(X), p(W), p(b), p(tgt), inp["ignore_index"], w.BT, w.H, w.V, dt, w.temperature,
+          cw, cb, p(logp), p(ws), ws.numel(), stream.cuda_stream)
+    ba = (p(X), p(W), p(b), p(tgt), inp["ignore_index"], w.BT, w.H, w.V, dt, w.temperature,
+          p(dlogp), cw, cb, True, p(dX), p(dW), p(db), p(ws), ws.numel(), stream.cuda_stream)
+
+    def step():
+        s = pkg.flkl_selective_logprob_forward(*fa)
+        if s == 0:
+            s = pkg.flkl_selective_logprob_backward(*ba)
+        if s != 0:
+            raise pkg.FlklError(s, "flkl_selective_logprob")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    if pkg.flkl_device_status(p(ws), stream.cuda_stream) != 0:
+        raise pkg.FlklError(4, "device status after the timed region")
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, peak_src = load_peaks()
+    flops = 2.0 * w.BT * w.H * w.V * (2 + (1 if cw else 0))
+    achieved = flops / (ms * 1e-3) / 1e12
+    # the oracle on the host cores: a bounded sample of rows, forward + backward
+    from oracle import selective_logprob, selective_logprob_backward
+    rows = min(args.cpu_sample_rows, w.BT)
+    host = make_inputs(w.with_(BT=rows, seed=123), device="cpu")
+    f = lambda t: None if t is None else t.float().numpy().astype(np.float64)
+    Xh, Wh, bh, th = f(host["X"]), f(host["W"]), f(host["b"]), host["target"].numpy()
+    t0 = time.perf_counter()
+    selective_logprob(Xh, Wh, bh, th, inp["ignore_index"], w.temperature)
+    selective_logprob_backward(Xh, Wh, bh, th, np.ones(rows), inp["ignore_index"],
+                               w.temperature, compute_dW=cw, compute_db=cb)
+    t_cpu = time.perf_counter() - t0
+    line = {
+        "metric": "selective log-prob fwd+bwd tokens/s", "value": round(w.BT / (ms * 1e-3), 1),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": name, "BT": w.BT, "H": w.H, "V": w.V, "compute_dW": cw,
+                   "compute_db": cb, "l2": "inputs larger than L2 (W), no flush"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": None, "scope": "whole step (counted FLOPs)",
+                     "peak_source": peak_src},
+        "cpu_baseline": {"value": round(rows / t_cpu, 2), "unit": "tokens/s",
+                         "cores": host_threads(), "kind": "oracle",
+                         "sample": f"{rows} rows of {name}, fp64 numpy, {t_cpu:.1f} s"},
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.op != "loss":
+    if a.op == "logprob":
+        run_logprob(a)
+    elif a.op != "loss":
         run_norm(a)
     elif a.impl == "reference":
         run_reference(a)
