@@ -574,7 +574,6 @@ class _SelectiveLogProbFunction(torch.autograd.Function):
             _ptr(ctx.ws), ctx.ws.numel(), st.cuda_stream)
         if s != FLKL_OK:
             raise FlklError(s, "flkl_selective_logprob_backward")
-        ctx.ws = None
         if dW is not None:
             dW = dW.to(W.dtype)
         if db is not None:
