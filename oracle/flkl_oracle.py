@@ -361,3 +361,86 @@ def selective_logprob_backward(X, W, b, target, dlogp, ignore_index=-100, temper
         if db is not None:
             db += G.sum(axis=0)
     return dict(dX=dX, dW=dW, db=db)
+
+
+def jsd_forward_backward(X, W, b, Xt, Wt, bt, shift_labels=None, ignore_index=-100,
+                         temperature=1.0, beta=0.5, reduction="batchmean", compute_dW=True,
+                         compute_db=False, dX_rows=None, dW_rows=None, row_block=256):
+    """Fused linear Jensen-Shannon divergence, fp64.
+
+    The FusedLinearKLDivLoss page names LigerFusedLinearJSD as the sibling
+    loss whose teacher side has its own projection; it prints no formula.
+    Reading used here (the generalized JSD): student P = softmax((X W^T +
+    b)/T), teacher Q = softmax((Xt Wt^T + bt)/T), M = beta P + (1 - beta) Q,
+
+        l_r = beta KL(P_r || M_r) + (1 - beta) KL(Q_r || M_r),
+
+    with 0 log 0 = 0, rows dropped by shift_labels == ignore_index, and the
+    divisors of the KL loss (batchmean: N_valid, mean: N_valid * V, sum: 1).
+    Only the student gets gradients:
+
+        d l_r / d z_rv = beta p_rv (log(p_rv / m_rv) - KL(P_r || M_r)) / T.
+    """
+    if reduction not in REDUCTIONS:
+        raise OracleError(f"reduction={reduction!r} is not supported")
+    if not (0.0 < beta < 1.0):
+        raise OracleError("beta must lie in (0, 1)")
+    if compute_db and b is None:
+        raise OracleError("compute_db needs a bias")
+    BT, H = np.shape(X)
+    V = np.shape(W)[0]
+    T = float(temperature)
+    valid = valid_rows(BT, shift_labels, ignore_index)
+    n_valid = int(valid.sum())
+    D = divisor(reduction, n_valid, V)
+    scale = 0.0 if n_valid == 0 else 1.0 / (T * D)
+    W64, b64 = _as64(W), _as64(b)
+    Wt64, bt64 = _as64(Wt), _as64(bt)
+    dx_sel = np.arange(BT) if dX_rows is None else np.asarray(dX_rows, dtype=np.int64)
+    dw_sel = None if not compute_dW else (np.arange(V) if dW_rows is None
+                                          else np.asarray(dW_rows, dtype=np.int64))
+    dX = np.zeros((len(dx_sel), H))
+    dW = None if dw_sel is None else np.zeros((len(dw_sel), H))
+    db = np.zeros(V) if compute_db else None
+    row_loss = np.zeros(BT)
+    dx_pos = {int(r): i for i, r in enumerate(dx_sel)}
+
+    def xlogy(x, y):
+        # x * log(x / y) with 0 log 0 = 0 (y > 0 wherever x > 0)
+        out = np.zeros_like(x)
+        nz = x > 0
+        out[nz] = x[nz] * np.log(x[nz] / y[nz])
+        return out
+
+    for r0 in range(0, BT, row_block):
+        r1 = min(BT, r0 + row_block)
+        Xc = _as64(X[r0:r1])
+        zs = Xc @ W64.T
+        if b64 is not None:
+            zs += b64
+        zt = _as64(Xt[r0:r1]) @ Wt64.T
+        if bt64 is not None:
+            zt += bt64
+        logp, _ = log_softmax_rows(zs / T)
+        logq, _ = log_softmax_rows(zt / T)
+        p, q = np.exp(logp), np.exp(logq)
+        m = beta * p + (1.0 - beta) * q
+        kl_pm = xlogy(p, m)
+        kl_qm = xlogy(q, m)
+        K = kl_pm.sum(axis=1)
+        keep = valid[r0:r1]
+        row_loss[r0:r1] = np.where(keep, beta * K + (1.0 - beta) * kl_qm.sum(axis=1), 0.0)
+        ell = np.zeros_like(p)
+        nz = p > 0
+        ell[nz] = np.log(p[nz] / m[nz])
+        G = beta * p * (ell - K[:, None]) * scale
+        G[~keep] = 0.0
+        here = [i for i in range(r0, r1) if i in dx_pos]
+        if here:
+            dX[[dx_pos[i] for i in here]] = G[np.asarray(here) - r0] @ W64
+        if dW is not None:
+            dW += G[:, dw_sel].T @ Xc
+        if db is not None:
+            db += G.sum(axis=0)
+    loss = 0.0 if n_valid == 0 else float(row_loss.sum() / D)
+    return dict(loss=loss, dX=dX, dW=dW, db=db, row_loss=row_loss, n_valid=n_valid, D=D)
