@@ -176,6 +176,29 @@ FLKL_API flkl_status flkl_selective_logprob_backward(
     int compute_dW, int compute_db, int accum_fp32, void* dX, void* dW, void* db,
     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Fused linear Jensen-Shannon divergence (the FusedLinearKLDivLoss page,
+ * Summary, names LigerFusedLinearJSD as the sibling loss whose teacher side
+ * has its own projection; the pages print no formula, the generalized JSD is
+ * the reading used).  Student P = softmax((X W^T + b)/T), teacher
+ * Q = softmax((Xt Wt^T + bt)/T), M = beta P + (1 - beta) Q:
+ *   loss = sum over kept rows of [beta KL(P||M) + (1 - beta) KL(Q||M)] / D
+ * with the divisors, row mask (shift_labels), outputs, flags and errors of
+ * flkl_forward_backward; only the student gets gradients,
+ *   dz_rv = beta p_rv (log(p_rv / m_rv) - KL(P_r||M_r)) / (T D).
+ *  Xt [BT, Ht], Wt [V, Ht], bt [V] (nullable): teacher hidden states and head,
+ *  `dtype` like X; Ht a multiple of 8 (bf16) or 4 (fp32).  0 < beta < 1.
+ *  workspace: flkl_jsd_workspace_size bytes (no BT x V buffer: two
+ *  staging blocks of one vocabulary chunk).  The probabilities of a chunk are
+ *  staged in the input dtype (bf16 on the tensor-core path). */
+FLKL_API size_t flkl_jsd_workspace_size(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype,
+                                        int compute_dW, int compute_db);
+FLKL_API flkl_status flkl_jsd_forward_backward(
+    const void* X, const void* W, const void* b, const void* Xt, const void* Wt, const void* bt,
+    const int64_t* shift_labels, int64_t ignore_index, int64_t BT, int64_t H, int64_t Ht,
+    int64_t V, int dtype, float temperature, float beta, int reduction, int compute_dW,
+    int compute_db, int accum_fp32, float* loss, void* dX, void* dW, void* db, void* workspace,
+    size_t workspace_bytes, void* stream);
+
 /* Data-parallel use: the batch is split by rows over ranks that share the
  * head W, b (the row sharding of the scope table's multi-GPU row).  Each rank
  * calls flkl_count_valid on its labels (or targets), all-reduces the int64

@@ -25,6 +25,8 @@ __all__ = [
     "flkl_norm_device_status", "flkl_count_valid", "flkl_forward_backward_dp",
     "flkl_ce_forward_backward_dp", "count_valid", "flkl_selective_logprob_forward",
     "flkl_selective_logprob_backward", "selective_logprob", "SelectiveLogProb",
+    "flkl_jsd_workspace_size", "flkl_jsd_forward_backward", "jsd_forward_backward",
+    "FusedLinearJSDLoss",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -97,6 +99,15 @@ def _lib():
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_int64, c.c_int64,
             c.c_int64, c.c_int, c.c_float, c.c_void_p, c.c_int, c.c_int, c.c_int, c.c_void_p,
             c.c_void_p, c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.flkl_jsd_workspace_size.restype = c.c_size_t
+        lib.flkl_jsd_workspace_size.argtypes = [c.c_int64, c.c_int64, c.c_int64, c.c_int64,
+                                                c.c_int, c.c_int, c.c_int]
+        lib.flkl_jsd_forward_backward.restype = c.c_int
+        lib.flkl_jsd_forward_backward.argtypes = [
+            c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+            c.c_int64, c.c_int64, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_float,
+            c.c_float, c.c_int, c.c_int, c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_void_p,
+            c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
         lib.flkl_count_valid.restype = c.c_int
         lib.flkl_count_valid.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p]
         lib.flkl_forward_backward_noalloc.restype = c.c_int
@@ -211,6 +222,23 @@ def flkl_selective_logprob_backward(X, W, b, target, ignore_index, BT, H, V, dty
         X, W, b, target, int(ignore_index), int(BT), int(H), int(V), int(dtype),
         float(temperature), dlogp, int(bool(compute_dW)), int(bool(compute_db)),
         int(bool(accum_fp32)), dX, dW, db, workspace, int(workspace_bytes), stream)
+
+
+def flkl_jsd_workspace_size(BT, H, Ht, V, dtype, compute_dW, compute_db) -> int:
+    return _lib().flkl_jsd_workspace_size(int(BT), int(H), int(Ht), int(V), int(dtype),
+                                          int(bool(compute_dW)), int(bool(compute_db)))
+
+
+def flkl_jsd_forward_backward(X, W, b, Xt, Wt, bt, shift_labels, ignore_index, BT, H, Ht, V,
+                              dtype, temperature, beta, reduction, compute_dW, compute_db,
+                              accum_fp32, loss, dX, dW, db, workspace, workspace_bytes,
+                              stream) -> int:
+    """The fused linear JSD entry point with raw pointers; returns the status."""
+    return _lib().flkl_jsd_forward_backward(
+        X, W, b, Xt, Wt, bt, shift_labels, int(ignore_index), int(BT), int(H), int(Ht), int(V),
+        int(dtype), float(temperature), float(beta), int(reduction), int(bool(compute_dW)),
+        int(bool(compute_db)), int(bool(accum_fp32)), loss, dX, dW, db, workspace,
+        int(workspace_bytes), stream)
 
 
 def flkl_norm_workspace_size(rows, H, compute_dW, compute_db) -> int:
@@ -499,6 +527,120 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
         if s != FLKL_OK:
             raise FlklError(s, "flkl_ce_forward_backward (device)")
     return {"loss": loss, "dX": dX, "dW": dW, "db": db, "workspace": workspace}
+
+
+def jsd_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor],
+                         Xt: torch.Tensor, Wt: torch.Tensor, bt: Optional[torch.Tensor] = None,
+                         shift_labels: Optional[torch.Tensor] = None, ignore_index: int = -100,
+                         temperature: float = 1.0, beta: float = 0.5,
+                         reduction: str = "batchmean", compute_dW: bool = True,
+                         compute_db: bool = False, accum_fp32: bool = True,
+                         workspace: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None,
+                         check_status: bool = False) -> dict:
+    """Fused linear Jensen-Shannon divergence between the student head
+    (X, W, b) and the teacher head (Xt, Wt, bt) in one call: the generalized
+    JSD with weight ``beta`` (M = beta P + (1 - beta) Q), loss and student
+    gradients; returns ``{"loss", "dX", "dW", "db", "workspace"}``."""
+    if reduction not in REDUCTIONS:
+        raise ValueError(f"unknown reduction {reduction!r}")
+    if X.dtype not in DTYPES:
+        raise ValueError(f"dtype {X.dtype} not supported (float32 or bfloat16)")
+    dev, dt = X.device, X.dtype
+    BT, H = X.shape
+    V = W.shape[0]
+    Ht = Xt.shape[1]
+    _check_dev("X", X, dt, (BT, H), dev)
+    _check_dev("W", W, dt, (V, H), dev)
+    _check_dev("Xt", Xt, dt, (BT, Ht), dev)
+    _check_dev("Wt", Wt, dt, (V, Ht), dev)
+    if b is not None:
+        _check_dev("b", b, dt, (V,), dev)
+    if bt is not None:
+        _check_dev("bt", bt, dt, (V,), dev)
+    if shift_labels is not None:
+        _check_dev("shift_labels", shift_labels, torch.int64, (BT,), dev)
+    compute_db = bool(compute_db and b is not None)
+    pdt = torch.float32 if (accum_fp32 or dt == torch.float32) else dt
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    dX = torch.empty_like(X)
+    dW = torch.empty((V, H), dtype=pdt, device=dev) if compute_dW else None
+    db = torch.empty((V,), dtype=pdt, device=dev) if compute_db else None
+    need = flkl_jsd_workspace_size(BT, H, Ht, V, DTYPES[dt], compute_dW, compute_db)
+    if need == 0:
+        raise FlklError(1, "flkl_jsd_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = stream if stream is not None else torch.cuda.current_stream(dev)
+    status = flkl_jsd_forward_backward(
+        _ptr(X), _ptr(W), _ptr(b), _ptr(Xt), _ptr(Wt), _ptr(bt), _ptr(shift_labels),
+        ignore_index, BT, H, Ht, V, DTYPES[dt], temperature, beta, REDUCTIONS[reduction],
+        compute_dW, compute_db, accum_fp32, _ptr(loss), _ptr(dX), _ptr(dW), _ptr(db),
+        _ptr(workspace), workspace.numel(), st.cuda_stream)
+    if status != FLKL_OK:
+        raise FlklError(status, "flkl_jsd_forward_backward")
+    if check_status:
+        s = flkl_device_status(_ptr(workspace), st.cuda_stream)
+        if s != FLKL_OK:
+            raise FlklError(s, "flkl_jsd_forward_backward (device)")
+    return {"loss": loss, "dX": dX, "dW": dW, "db": db, "workspace": workspace}
+
+
+class _FusedLinearJSDFunction(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, X, W, b, Xt, Wt, bt, shift_labels, ignore_index, temperature, beta,
+                reduction, accum_fp32):
+        r = jsd_forward_backward(
+            X.contiguous(), W.contiguous(), None if b is None else b.contiguous(),
+            Xt.contiguous(), Wt.contiguous(), None if bt is None else bt.contiguous(),
+            None if shift_labels is None else shift_labels.contiguous(), ignore_index,
+            temperature, beta, reduction, compute_dW=ctx.needs_input_grad[1],
+            compute_db=b is not None and ctx.needs_input_grad[2], accum_fp32=accum_fp32)
+        ctx.save_for_backward(r["dX"], r["dW"], r["db"])
+        ctx.w_dtype = W.dtype
+        return r["loss"]
+
+    @staticmethod
+    def backward(ctx, grad_out):
+        dX, dW, db = ctx.saved_tensors
+        if not bool((grad_out == 1).all()):
+            dX = dX * grad_out.to(dX.dtype)
+            dW = None if dW is None else dW * grad_out.to(dW.dtype)
+            db = None if db is None else db * grad_out.to(db.dtype)
+        if dW is not None:
+            dW = dW.to(ctx.w_dtype)
+        if db is not None:
+            db = db.to(ctx.w_dtype)
+        return dX, dW, db, None, None, None, None, None, None, None, None, None
+
+
+class FusedLinearJSDLoss(torch.nn.Module):
+    """Fused linear generalized Jensen-Shannon divergence between a student
+    head and a teacher head (the teacher gets no gradient), gradient in
+    forward: ``forward(student_weight, student_input, teacher_input,
+    teacher_weight, shift_labels=None, student_bias=None, teacher_bias=None)``.
+    """
+
+    def __init__(self, beta: float = 0.5, ignore_index: int = -100,
+                 temperature: float = 1.0, reduction: str = "batchmean",
+                 accum_dtype: Optional[torch.dtype] = None):
+        super().__init__()
+        if not 0.0 < beta < 1.0:
+            raise ValueError("beta must lie in (0, 1)")
+        if reduction not in ("batchmean", "mean", "sum"):
+            raise ValueError(f"reduction {reduction!r} is not supported")
+        self.beta, self.ignore_index, self.temperature = beta, ignore_index, temperature
+        self.reduction = reduction
+        self.accum_fp32 = accum_dtype == torch.float32
+
+    def forward(self, student_weight, student_input, teacher_input, teacher_weight,
+                shift_labels=None, student_bias=None, teacher_bias=None):
+        return _FusedLinearJSDFunction.apply(student_input, student_weight, student_bias,
+                                             teacher_input.detach(), teacher_weight.detach(),
+                                             None if teacher_bias is None
+                                             else teacher_bias.detach(),
+                                             shift_labels, self.ignore_index, self.temperature,
+                                             self.beta, self.reduction, self.accum_fp32)
 
 
 def count_valid(labels: Optional[torch.Tensor], BT: int, ignore_index: int = -100,

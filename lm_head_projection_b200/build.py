@@ -15,7 +15,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "_flkl.so")
 SOURCES = ["flkl_api.cu", "norm_api.cu"]
-HEADERS = ["ptx.cuh", "tc_gemm.cuh", "row_kernels.cuh", "simt_f32.cuh", "norm_bwd.cuh"]
+HEADERS = ["ptx.cuh", "tc_gemm.cuh", "row_kernels.cuh", "simt_f32.cuh", "norm_bwd.cuh",
+           "jsd_kernels.cuh"]
 
 
 def nvcc_path() -> str:

@@ -21,6 +21,7 @@
 #include <mutex>
 
 #include "../../include/flkl.h"
+#include "jsd_kernels.cuh"
 #include "row_kernels.cuh"
 #include "simt_f32.cuh"
 #include "tc_gemm.cuh"
@@ -475,6 +476,284 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
   return FLKL_OK;
 }
 
+// ------------------------------------------------------------------ JSD
+// Fused linear Jensen-Shannon divergence (flkl_jsd_forward_backward): the
+// same GEMM kernels, twice per side.  Sequence:
+//   statistics passes of the teacher and of the student (log-sum-exps),
+//   per vocabulary chunk: both sides' probabilities into staging, then the
+//     row sums K = KL(P||M) and l (k_jsd_rows);  loss = sum of kept l / D,
+//   per vocabulary chunk again: both sides' probabilities, the gradient block
+//     G (k_jsd_grad, written over the student's probabilities, with db column
+//     partials), then dX(c) and dW(c).
+struct JsdPlan {
+  bool tc;
+  long long m_tiles, n_tiles, n_stat, Vc, nchunks, db_groups, n_counters;
+  size_t off_cnt, off_st, off_rows, off_tgt, off_P, off_Q, off_G, off_dx, off_db, total;
+};
+
+constexpr int kJsdRows = 10;  // fp32 row arrays in the workspace
+
+bool make_jsd_plan(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype, int compute_db,
+                   JsdPlan& p) {
+  if (BT < 0 || H < 1 || Ht < 1 || V < 1) return false;
+  if (BT >= (int64_t(1) << 31) || H >= (int64_t(1) << 31) || Ht >= (int64_t(1) << 31) ||
+      V >= (int64_t(1) << 31))
+    return false;
+  if (dtype != FLKL_DTYPE_F32 && dtype != FLKL_DTYPE_BF16) return false;
+  p.tc = dtype == FLKL_DTYPE_BF16;
+  const int tile = p.tc ? TC_BN : ST_T;
+  const size_t elem = p.tc ? 2 : 4;
+  p.m_tiles = cdiv(BT, p.tc ? TC_BM : ST_T);
+  p.n_tiles = cdiv(V, tile);
+  p.n_stat = p.tc ? cdiv(V, TC_EPI_COLS) : p.n_tiles;
+  long long vc = cdiv(cdiv(V, 8), tile) * tile;
+  if (BT > 0) {
+    long long cap = static_cast<long long>(kStagingBudget / (size_t(BT) * elem));
+    cap = (cap / tile) * tile;
+    vc = std::min(vc, std::max<long long>(cap, tile));
+  }
+  vc = std::min(vc, p.n_tiles * tile);
+  p.Vc = vc;
+  p.nchunks = cdiv(V, vc);
+  p.db_groups = cdiv(BT, kJsdRowGroup);
+  p.n_counters = 2 + 5 * p.nchunks;
+  size_t off = align256(sizeof(DevCtl));
+  p.off_cnt = off;
+  off += align256(size_t(p.n_counters) * 4);
+  p.off_st = off;
+  off += align256(size_t(5) * p.n_stat * BT * 4);
+  p.off_rows = off;
+  off += align256(size_t(kJsdRows) * BT * 4);
+  p.off_tgt = off;
+  off += align256(size_t(BT) * 8);
+  // student and teacher probabilities of one chunk; the gradient block
+  // overwrites the student's in place
+  const size_t stage = align256(size_t(BT) * vc * elem);
+  p.off_P = off;
+  p.off_Q = off + stage;
+  p.off_G = off;
+  off += 2 * stage;
+  p.off_dx = off;
+  if (p.nchunks > 1) off += align256(size_t(BT) * H * 4);
+  p.off_db = off;
+  if (compute_db) off += align256(size_t(p.db_groups) * V * 4);
+  p.total = off;
+  return true;
+}
+
+struct JsdRows {
+  float *lse2_t, *lse2_s, *scrS, *scrQ, *scrL, *K, *L, *rowscale, *ones, *zeros;
+};
+
+JsdRows jsd_rows(float* rows, int BT) {
+  JsdRows r;
+  float** f[kJsdRows] = {&r.lse2_t, &r.lse2_s, &r.scrS, &r.scrQ, &r.scrL,
+                         &r.K,      &r.L,      &r.rowscale, &r.ones, &r.zeros};
+  for (int i = 0; i < kJsdRows; ++i) *f[i] = rows + static_cast<size_t>(i) * BT;
+  return r;
+}
+
+cudaError_t jsd_prepare_rows(const JsdRows& R, int64_t* nt, int BT, int V, cudaStream_t st) {
+  const unsigned g = static_cast<unsigned>(cdiv(BT, 256));
+  // "no target" for the cross-entropy mode of the GEMM epilogues: index V
+  k_fill_i64<<<g, 256, 0, st>>>(nt, BT, V);
+  k_fill_f32<<<g, 256, 0, st>>>(R.ones, BT, 1.f);
+  k_fill_f32<<<g, 256, 0, st>>>(R.zeros, BT, 0.f);
+  return cudaGetLastError();
+}
+
+flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bfloat16* W,
+                       const __nv_bfloat16* b, const __nv_bfloat16* Xt, const __nv_bfloat16* Wt,
+                       const __nv_bfloat16* bt, const int64_t* labels, long long ignore_index,
+                       int BT, int H, int Ht, int V, float T, float beta, int compute_dW,
+                       int compute_db, int accum_fp32, float* loss, __nv_bfloat16* dX, void* dW,
+                       void* db, uint8_t* ws, cudaStream_t st) {
+  DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
+  int* counters = reinterpret_cast<int*>(ws + P.off_cnt);
+  float* stats = reinterpret_cast<float*>(ws + P.off_st);
+  const JsdRows R = jsd_rows(reinterpret_cast<float*>(ws + P.off_rows), BT);
+  int64_t* nt = reinterpret_cast<int64_t*>(ws + P.off_tgt);
+  __nv_bfloat16* Pb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_P);
+  __nv_bfloat16* Qb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_Q);
+  __nv_bfloat16* Gb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_G);
+  float* dxpart = reinterpret_cast<float*>(ws + P.off_dx);
+  float* dbpart = compute_db ? reinterpret_cast<float*>(ws + P.off_db) : nullptr;
+  const float t_scale = 1.4426950408889634f / T;
+  const int ldg = static_cast<int>(P.Vc);
+  FLKL_CUDA(jsd_prepare_rows(R, nt, BT, V, st));
+
+  Operand mX_k, mW_k, mX_mn, mW_mn, mXt_k, mWt_k;
+  if (!make_operand(&mX_k, X, H, BT, H, false) || !make_operand(&mW_k, W, H, V, H, false) ||
+      !make_operand(&mX_mn, X, H, BT, H, true) || !make_operand(&mW_mn, W, H, V, H, true) ||
+      !make_operand(&mXt_k, Xt, Ht, BT, Ht, false) || !make_operand(&mWt_k, Wt, Ht, V, Ht, false))
+    return FLKL_ERR_CUDA;
+  int counter = 0;
+  auto new_launch = [&]() {
+    TcLaunch L{};
+    L.counter = counters + counter++;
+    L.err_flag = &ctl->err;
+    L.wait_limit_ns = g_wait_limit_ns;
+    return L;
+  };
+  auto chunk_c0 = [&](long long c) { return static_cast<int>(c * P.Vc); };
+  auto chunk_w = [&](long long c) {
+    return static_cast<int>(std::min<long long>(P.Vc, V - c * P.Vc));
+  };
+  // log-sum-exp of one side: statistics pass (no teacher) + merge
+  auto side_lse = [&](const Operand& mA, const Operand& mB, int Hk, const __nv_bfloat16* bias,
+                      float* lse2) -> cudaError_t {
+    TcLaunch L = new_launch();
+    TcMaps maps{};
+    L.stats = EpiStats::Params{nullptr, bias, BT, V, t_scale, 0.f, stats,
+                               static_cast<long long>(P.n_stat) * BT, nt};
+    add_problem(L, maps, KIND_STATS, BT, V, Hk, 1, mA, mB);
+    cudaError_t e = launch_group(maps, L, st);
+    if (e != cudaSuccess) return e;
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
+        stats, static_cast<int>(P.n_stat), BT, nullptr, ignore_index, 1.f / T, ctl, lse2, R.scrS,
+        R.scrQ, R.scrL);
+    return cudaGetLastError();
+  };
+  // probabilities of one side over chunk c into `out` (the pass-2 epilogue
+  // with coefficients 1 and 0 and no teacher)
+  auto side_probs = [&](const Operand& mA, const Operand& mB, int Hk,
+                        const __nv_bfloat16* bias, const float* lse2, __nv_bfloat16* out,
+                        long long c) -> cudaError_t {
+    TcLaunch L = new_launch();
+    TcMaps maps{};
+    const int c0 = chunk_c0(c);
+    L.grad = EpiGrad::Params{nullptr, bias, BT,     V,       c0,      ldg,     out,
+                             t_scale, lse2, R.ones, R.zeros, nullptr, nt};
+    add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), Hk, 1, mA, mB, 0, c0, 0);
+    return launch_group(maps, L, st);
+  };
+
+  FLKL_CUDA(side_lse(mXt_k, mWt_k, Ht, bt, R.lse2_t));
+  FLKL_CUDA(side_lse(mX_k, mW_k, H, b, R.lse2_s));
+  k_jsd_init_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
+      labels, BT, ignore_index, ctl, R.rowscale, R.K, R.L);
+  FLKL_CUDA(cudaGetLastError());
+  for (long long c = 0; c < P.nchunks; ++c) {
+    FLKL_CUDA(side_probs(mXt_k, mWt_k, Ht, bt, R.lse2_t, Qb, c));
+    FLKL_CUDA(side_probs(mX_k, mW_k, H, b, R.lse2_s, Pb, c));
+    k_jsd_rows<__nv_bfloat16><<<static_cast<unsigned>(cdiv(int64_t(BT) * 32, 256)), 256, 0, st>>>(
+        Pb, Qb, ldg, BT, chunk_w(c), beta, R.K, R.L);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  k_jsd_row_loss<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(R.L, R.rowscale, BT,
+                                                                         R.scrL);
+  k_loss<<<1, 1024, 0, st>>>(R.scrL, BT, ctl, loss);
+  FLKL_CUDA(cudaGetLastError());
+  for (long long c = 0; c < P.nchunks; ++c) {
+    const int c0 = chunk_c0(c), Vw = chunk_w(c);
+    FLKL_CUDA(side_probs(mXt_k, mWt_k, Ht, bt, R.lse2_t, Qb, c));
+    FLKL_CUDA(side_probs(mX_k, mW_k, H, b, R.lse2_s, Pb, c));
+    k_jsd_grad<__nv_bfloat16>
+        <<<dim3(static_cast<unsigned>(cdiv(Vw, 256)), static_cast<unsigned>(P.db_groups)), 256,
+           0, st>>>(Pb, Qb, ldg, BT, Vw, c0, V, beta, R.K, R.rowscale, Gb, dbpart);
+    FLKL_CUDA(cudaGetLastError());
+    Operand mG_k, mG_mn;
+    if (!make_operand(&mG_k, Gb, Vw, BT, ldg, false) || !make_operand(&mG_mn, Gb, Vw, BT, ldg, true))
+      return FLKL_ERR_CUDA;
+    TcLaunch L = new_launch();
+    TcMaps maps{};
+    const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
+    L.dx = EpiAccumRows::Params{dxpart, dX, H, BT, H, mode};
+    add_problem(L, maps, KIND_DX, BT, H, Vw, 0, mG_k, mW_mn, 0, 0, c0);
+    if (compute_dW) {
+      L.dw = EpiStoreRows::Params{dW, H, Vw, H, c0, accum_fp32};
+      add_problem(L, maps, KIND_DW, Vw, H, BT, 1, mG_mn, mX_mn);
+    }
+    FLKL_CUDA(launch_group(maps, L, st));
+  }
+  if (compute_db) {
+    k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
+        dbpart, static_cast<int>(P.db_groups), V, db, accum_fp32);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  return FLKL_OK;
+}
+
+flkl_status run_jsd_f32(const JsdPlan& P, const float* X, const float* W, const float* b,
+                        const float* Xt, const float* Wt, const float* bt, const int64_t* labels,
+                        long long ignore_index, int BT, int H, int Ht, int V, float T, float beta,
+                        int compute_dW, int compute_db, float* loss, float* dX, float* dW,
+                        float* db, uint8_t* ws, cudaStream_t st) {
+  DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
+  float* stats = reinterpret_cast<float*>(ws + P.off_st);
+  const JsdRows R = jsd_rows(reinterpret_cast<float*>(ws + P.off_rows), BT);
+  int64_t* nt = reinterpret_cast<int64_t*>(ws + P.off_tgt);
+  float* Pb = reinterpret_cast<float*>(ws + P.off_P);
+  float* Qb = reinterpret_cast<float*>(ws + P.off_Q);
+  float* Gb = reinterpret_cast<float*>(ws + P.off_G);
+  float* dxpart = reinterpret_cast<float*>(ws + P.off_dx);
+  float* dbpart = compute_db ? reinterpret_cast<float*>(ws + P.off_db) : nullptr;
+  const float t_scale = 1.4426950408889634f / T;
+  const int ldg = static_cast<int>(P.Vc);
+  const unsigned mt = static_cast<unsigned>(P.m_tiles);
+  FLKL_CUDA(jsd_prepare_rows(R, nt, BT, V, st));
+  auto side_lse = [&](const float* A, const float* B, int Hk, const float* bias, float* lse2) {
+    k_simt_stats<<<dim3(static_cast<unsigned>(P.n_tiles), mt), 256, 0, st>>>(
+        A, B, bias, nullptr, BT, Hk, V, t_scale, 0.f, stats,
+        static_cast<long long>(P.n_tiles) * BT, nt);
+    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
+        stats, static_cast<int>(P.n_stat), BT, nullptr, ignore_index, 1.f / T, ctl, lse2, R.scrS,
+        R.scrQ, R.scrL);
+    return cudaGetLastError();
+  };
+  auto side_probs = [&](const float* A, const float* B, int Hk, const float* bias,
+                        const float* lse2, float* out, int c0, int Vw) {
+    k_simt_grad<<<dim3(static_cast<unsigned>(cdiv(Vw, ST_T)), mt), 256, 0, st>>>(
+        A, B, bias, nullptr, BT, Hk, V, c0, Vw, t_scale, lse2, R.ones, R.zeros, out, ldg,
+        nullptr, nt);
+    return cudaGetLastError();
+  };
+  FLKL_CUDA(side_lse(Xt, Wt, Ht, bt, R.lse2_t));
+  FLKL_CUDA(side_lse(X, W, H, b, R.lse2_s));
+  k_jsd_init_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
+      labels, BT, ignore_index, ctl, R.rowscale, R.K, R.L);
+  FLKL_CUDA(cudaGetLastError());
+  for (long long c = 0; c < P.nchunks; ++c) {
+    const int c0 = static_cast<int>(c * P.Vc);
+    const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
+    FLKL_CUDA(side_probs(Xt, Wt, Ht, bt, R.lse2_t, Qb, c0, Vw));
+    FLKL_CUDA(side_probs(X, W, H, b, R.lse2_s, Pb, c0, Vw));
+    k_jsd_rows<float><<<static_cast<unsigned>(cdiv(int64_t(BT) * 32, 256)), 256, 0, st>>>(
+        Pb, Qb, ldg, BT, Vw, beta, R.K, R.L);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  k_jsd_row_loss<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(R.L, R.rowscale, BT,
+                                                                         R.scrL);
+  k_loss<<<1, 1024, 0, st>>>(R.scrL, BT, ctl, loss);
+  FLKL_CUDA(cudaGetLastError());
+  for (long long c = 0; c < P.nchunks; ++c) {
+    const int c0 = static_cast<int>(c * P.Vc);
+    const int Vw = static_cast<int>(std::min<long long>(P.Vc, V - c0));
+    FLKL_CUDA(side_probs(Xt, Wt, Ht, bt, R.lse2_t, Qb, c0, Vw));
+    FLKL_CUDA(side_probs(X, W, H, b, R.lse2_s, Pb, c0, Vw));
+    k_jsd_grad<float>
+        <<<dim3(static_cast<unsigned>(cdiv(Vw, 256)), static_cast<unsigned>(P.db_groups)), 256,
+           0, st>>>(Pb, Qb, ldg, BT, Vw, c0, V, beta, R.K, R.rowscale, Gb, dbpart);
+    FLKL_CUDA(cudaGetLastError());
+    if (compute_dW) {
+      k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)),
+                             static_cast<unsigned>(cdiv(Vw, ST_T))),
+                        256, 0, st>>>(Gb, 1, ldg, X, 1, H, Vw, H, BT, nullptr, dW, H, c0, 4);
+      FLKL_CUDA(cudaGetLastError());
+    }
+    const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
+    k_simt_gemm_out<<<dim3(static_cast<unsigned>(cdiv(H, ST_T)), mt), 256, 0, st>>>(
+        Gb, ldg, 1, W + static_cast<size_t>(c0) * H, 1, H, BT, H, Vw, dxpart, dX, H, 0, mode);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  if (compute_db) {
+    k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
+        dbpart, static_cast<int>(P.db_groups), V, db, 1);
+    FLKL_CUDA(cudaGetLastError());
+  }
+  return FLKL_OK;
+}
+
 __global__ void k_wait_selftest(int* status, unsigned long long limit_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -626,6 +905,76 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
                  st, rec, target, ph);
 }
 
+flkl_status jsd_impl(const void* X, const void* W, const void* b, const void* Xt, const void* Wt,
+                     const void* bt, const int64_t* shift_labels, int64_t ignore_index,
+                     int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype, float temperature,
+                     float beta, int reduction, int compute_dW, int compute_db, int accum_fp32,
+                     float* loss, void* dX, void* dW, void* db, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  if (dtype != FLKL_DTYPE_F32 && dtype != FLKL_DTYPE_BF16) return FLKL_ERR_INVALID_ARG;
+  if (reduction == FLKL_REDUCTION_NONE) return FLKL_ERR_UNSUPPORTED;
+  if (reduction < FLKL_REDUCTION_BATCHMEAN || reduction > FLKL_REDUCTION_SUM)
+    return FLKL_ERR_INVALID_ARG;
+  if (!(temperature > 0.f) || !(temperature < INFINITY)) return FLKL_ERR_INVALID_ARG;
+  if (!(beta > 0.f) || !(beta < 1.f)) return FLKL_ERR_INVALID_ARG;
+  if (BT < 0 || H < 1 || Ht < 1 || V < 1) return FLKL_ERR_INVALID_ARG;
+  if (BT >= (int64_t(1) << 31) || H >= (int64_t(1) << 31) || Ht >= (int64_t(1) << 31) ||
+      V >= (int64_t(1) << 31))
+    return FLKL_ERR_UNSUPPORTED;
+  const int vec = dtype == FLKL_DTYPE_BF16 ? 8 : 4;
+  if (H % vec != 0 || Ht % vec != 0 || V % vec != 0) return FLKL_ERR_UNSUPPORTED;
+  if (W == nullptr || Wt == nullptr || loss == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (BT > 0 && (X == nullptr || Xt == nullptr || dX == nullptr)) return FLKL_ERR_INVALID_ARG;
+  if ((compute_dW != 0) != (dW != nullptr)) return FLKL_ERR_INVALID_ARG;
+  if ((compute_db != 0) != (db != nullptr)) return FLKL_ERR_INVALID_ARG;
+  if (compute_db && b == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(b) || !aligned16(Xt) || !aligned16(Wt) ||
+      !aligned16(bt) || !aligned16(dX) || !aligned16(dW) || !aligned16(db) ||
+      (reinterpret_cast<uintptr_t>(shift_labels) & 7u) || (reinterpret_cast<uintptr_t>(loss) & 3u))
+    return FLKL_ERR_UNSUPPORTED;
+  JsdPlan P;
+  if (!make_jsd_plan(BT, H, Ht, V, dtype, compute_db, P)) return FLKL_ERR_INVALID_ARG;
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < P.total)
+    return FLKL_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int bt_ = static_cast<int>(BT), h = static_cast<int>(H), ht = static_cast<int>(Ht),
+            v = static_cast<int>(V);
+  k_prepare<<<1, 1024, 0, st>>>(shift_labels, bt_, static_cast<long long>(ignore_index),
+                                reduction, v, temperature, reinterpret_cast<DevCtl*>(ws),
+                                reinterpret_cast<int*>(ws + P.off_cnt),
+                                static_cast<int>(P.n_counters), nullptr);
+  FLKL_CUDA(cudaGetLastError());
+  if (BT == 0) {
+    k_zero<<<1, 32, 0, st>>>(loss, sizeof(float));
+    const size_t pe = (dtype == FLKL_DTYPE_F32 || accum_fp32) ? 4 : 2;
+    if (compute_dW) {
+      const size_t bytes = size_t(V) * H * pe;
+      k_zero<<<static_cast<unsigned>(cdiv(bytes, 16 * 256)), 256, 0, st>>>(dW, bytes);
+    }
+    if (compute_db) {
+      const size_t bytes = size_t(V) * pe;
+      k_zero<<<static_cast<unsigned>(cdiv(bytes, 16 * 256)), 256, 0, st>>>(db, bytes);
+    }
+    return cudaGetLastError() == cudaSuccess ? FLKL_OK : FLKL_ERR_CUDA;
+  }
+  if (P.tc)
+    return run_jsd_tc(P, static_cast<const __nv_bfloat16*>(X),
+                      static_cast<const __nv_bfloat16*>(W), static_cast<const __nv_bfloat16*>(b),
+                      static_cast<const __nv_bfloat16*>(Xt),
+                      static_cast<const __nv_bfloat16*>(Wt),
+                      static_cast<const __nv_bfloat16*>(bt), shift_labels, ignore_index, bt_, h,
+                      ht, v, temperature, beta, compute_dW, compute_db, accum_fp32, loss,
+                      static_cast<__nv_bfloat16*>(dX), dW, db, ws, st);
+  return run_jsd_f32(P, static_cast<const float*>(X), static_cast<const float*>(W),
+                     static_cast<const float*>(b), static_cast<const float*>(Xt),
+                     static_cast<const float*>(Wt), static_cast<const float*>(bt), shift_labels,
+                     ignore_index, bt_, h, ht, v, temperature, beta, compute_dW, compute_db, loss,
+                     static_cast<float*>(dX), static_cast<float*>(dW), static_cast<float*>(db),
+                     ws, st);
+}
+
 // Fixed scratch of flkl_forward_backward_noalloc (see flkl.h): part of the
 // library's device image, so it exists on every device that loads the
 // library, without any allocation call.
@@ -745,6 +1094,27 @@ flkl_status flkl_ce_forward_backward_dp(const void* X, const void* W, const void
                                temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
                                BT > 0 ? target : nullptr, n_valid_total);
+}
+
+size_t flkl_jsd_workspace_size(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype,
+                                int compute_dW, int compute_db) {
+  (void)compute_dW;
+  JsdPlan p;
+  if (!make_jsd_plan(BT, H, Ht, V, dtype, compute_db, p)) return 0;
+  return p.total;
+}
+
+flkl_status flkl_jsd_forward_backward(const void* X, const void* W, const void* b, const void* Xt,
+                                      const void* Wt, const void* bt,
+                                      const int64_t* shift_labels, int64_t ignore_index,
+                                      int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype,
+                                      float temperature, float beta, int reduction,
+                                      int compute_dW, int compute_db, int accum_fp32,
+                                      float* loss, void* dX, void* dW, void* db,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  return jsd_impl(X, W, b, Xt, Wt, bt, shift_labels, ignore_index, BT, H, Ht, V, dtype,
+                  temperature, beta, reduction, compute_dW, compute_db, accum_fp32, loss, dX, dW,
+                  db, workspace, workspace_bytes, stream);
 }
 
 flkl_status flkl_selective_logprob_forward(const void* X, const void* W, const void* b,

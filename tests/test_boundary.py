@@ -218,3 +218,26 @@ def test_selective_logprob_entries_check_their_arguments():
     assert bwd(dX=None) == INVALID
     assert bwd(dW=None) == INVALID               # compute_dW without dW
     assert bwd(H=60) == UNSUPPORTED
+
+
+@no_gpu
+def test_jsd_entry_checks_its_arguments():
+    def jsd(**kw):
+        a = dict(X=P, W=P, b=None, Xt=P, Wt=P, bt=None, shift_labels=None, ignore_index=-100,
+                 BT=64, H=64, Ht=32, V=64, dtype=1, temperature=1.0, beta=0.5, reduction=0,
+                 compute_dW=1, compute_db=0, accum_fp32=1, loss=P, dX=P, dW=P, db=None,
+                 workspace=P, workspace_bytes=1 << 30, stream=None)
+        a.update(kw)
+        return pkg.flkl_jsd_forward_backward(**a)
+    assert jsd(beta=0.0) == INVALID
+    assert jsd(beta=1.0) == INVALID
+    assert jsd(beta=float("nan")) == INVALID
+    assert jsd(reduction=3) == UNSUPPORTED
+    assert jsd(Xt=None) == INVALID
+    assert jsd(Wt=None) == INVALID
+    assert jsd(Ht=36) == UNSUPPORTED          # bf16 teacher rows: multiple of 8
+    assert jsd(bt=P + 8) == UNSUPPORTED
+    assert jsd(compute_db=1, db=P) == INVALID  # db needs a bias
+    assert jsd(workspace_bytes=100) == WORKSPACE
+    need = pkg.flkl_jsd_workspace_size(1024, 4096, 4096, 128256, 1, 1, 0)
+    assert 0 < need < 1024 * 128256 * 2 // 2   # no BT x V buffer
