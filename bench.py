@@ -104,10 +104,11 @@ def parse():
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="loss",
-                    choices=["loss", "rms_norm", "layer_norm", "logprob"],
+                    choices=["loss", "rms_norm", "layer_norm", "logprob", "jsd"],
                     help="loss: the fused linear KL / CE loss (default); rms_norm / "
                          "layer_norm: the norm backward with frozen-parameter flags; logprob: "
-                         "selective log-probability forward + backward on a CE workload")
+                         "selective log-probability forward + backward on a CE workload; "
+                         "jsd: fused linear JSD with a teacher head of the same shape")
     ap.add_argument("--norm-shape", default="8192x8192", help="ROWSxH for --op *_norm")
     ap.add_argument("--norm-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--frozen", action="store_true", help="norm weight (and bias) frozen")
@@ -699,9 +700,90 @@ def run_logprob(args):
     print(json.dumps(line), flush=True)
 
 
+def run_jsd(args):
+    """Fused linear JSD on one GPU: the headline student head (bf16 BT=1024,
+    H=4096, V=128256, dW) against a teacher head of the same shape (its own
+    hidden states and weights); CUDA events around exactly K calls."""
+    import numpy as np
+
+    import lm_head_projection_b200 as pkg
+    from lm_head_projection_b200.workloads import WORKLOADS
+
+    w = WORKLOADS["bf16_bt1024_h4096_v128256"]
+    dev = torch.device("cuda", 0)
+    inp = make_inputs(w, device=dev)
+    tw = w.with_(seed=w.seed + 1000)
+    tin = make_inputs(tw, device=dev)
+    X, W, Xt, Wt = inp["X"], inp["W"], tin["X"], tin["W"]
+    beta = 0.5
+    r0 = pkg.jsd_forward_backward(X, W, None, Xt, Wt, None, beta=beta, compute_dW=True,
+                                  check_status=True)
+    ws = r0["workspace"]
+    p = lambda t: None if t is None else t.data_ptr()
+    stream = torch.cuda.current_stream(dev)
+    a = (p(X), p(W), None, p(Xt), p(Wt), None, None, -100, w.BT, w.H, w.H, w.V, 1, 1.0, beta,
+         0, True, False, True, p(r0["loss"]), p(r0["dX"]), p(r0["dW"]), None, p(ws),
+         ws.numel(), stream.cuda_stream)
+
+    def step():
+        s = pkg.flkl_jsd_forward_backward(*a)
+        if s != 0:
+            raise pkg.FlklError(s, "flkl_jsd_forward_backward")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    if pkg.flkl_device_status(p(ws), stream.cuda_stream) != 0:
+        raise pkg.FlklError(4, "device status after the timed region")
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks, peak_src = load_peaks()
+    # counted: teacher and student logits, dX and dW; executed: 8 such GEMMs
+    counted = 2.0 * w.BT * w.V * w.H * 4
+    achieved = counted / (ms * 1e-3) / 1e12
+    from oracle import jsd_forward_backward as oracle_jsd
+    rows = min(args.cpu_sample_rows, 256)
+    f = lambda t: t[:rows].float().cpu().numpy().astype(np.float64)
+    Wh, Wth = W.float().cpu().numpy().astype(np.float64), Wt.float().cpu().numpy().astype(
+        np.float64)
+    t0 = time.perf_counter()
+    oracle_jsd(f(X), Wh, None, f(Xt), Wth, None, beta=beta, compute_dW=True)
+    t_cpu = time.perf_counter() - t0
+    line = {
+        "metric": "fused linear JSD fwd+bwd tokens/s", "value": round(w.BT / (ms * 1e-3), 1),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "jsd_bf16_bt1024_h4096_ht4096_v128256", "BT": w.BT, "H": w.H,
+                   "Ht": w.H, "V": w.V, "beta": beta, "compute_dW": True,
+                   "l2": "inputs larger than L2 (W, Wt), no flush"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": None,
+                     "scope": "whole call; counted = teacher + student logits, dX, dW "
+                              "(8 GEMMs of that size run)", "peak_source": peak_src},
+        "cpu_baseline": {"value": round(rows / t_cpu, 2), "unit": "tokens/s",
+                         "cores": host_threads(), "kind": "oracle",
+                         "sample": f"{rows} rows, fp64 numpy, {t_cpu:.1f} s"},
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.op == "logprob":
+    if a.op == "jsd":
+        run_jsd(a)
+    elif a.op == "logprob":
         run_logprob(a)
     elif a.op != "loss":
         run_norm(a)
