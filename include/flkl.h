@@ -22,6 +22,13 @@
  * library recomputes them tile by tile in two passes and stages only a
  * bounded BT x Vc block of G (Vc <= V/8, rounded up to the tile width).
  *
+ * Declared below, besides that call: the same path with a one-hot teacher
+ * (cross-entropy) and as per-token log-probabilities with a separate backward
+ * (selective log-probability), the Jensen-Shannon divergence against a
+ * teacher head, a data-parallel form (whole-batch divisor), RMSNorm /
+ * LayerNorm backward with frozen-parameter flags, an allocation-free variant,
+ * workspace sizes, status and wait-limit helpers.
+ *
  * Conventions for every entry point:
  *  - Pointers named "device" are CUDA device pointers on the current device;
  *    the caller owns and allocates all of them (inputs, outputs, workspace).
