@@ -34,6 +34,13 @@ Readings where the pages are silent (each also listed in the design notes):
 5. The bias is added before dividing by T.
 6. Only equality of a shift label with ignore_index matters.
 
+Also here, each from its own definition (see the function docstrings): the
+cross-entropy special case (one-hot teacher), the per-token selective
+log-probability and its backward, and the generalized Jensen-Shannon
+divergence against a teacher head.  Every function is pinned by tests that
+do not restate it (library routines, closed forms, invariants, finite
+differences); none is unpinned.
+
 Everything runs in float64 on the exact input values (bf16 inputs are upcast).
 Rows are processed in blocks so that no BT x V fp64 array is held; the block
 size changes only summation order.
