@@ -233,6 +233,22 @@ FLKL_API flkl_status flkl_ce_forward_backward_dp(
     int compute_dW, int compute_db, int accum_fp32, float* loss, void* dX, void* dW, void* db,
     void* workspace, size_t workspace_bytes, void* stream, const int64_t* n_valid_total);
 
+/* Gradient-in-forward scaling for autograd (the FusedLinearKLDivLoss page,
+ * Details, bullet 3: the gradients come from the forward call; the backward
+ * only applies the incoming gradient of the loss):
+ *   dst[i] = dst_dtype(src[i] * *scale),  0 <= i < n
+ * with the multiplication skipped when *scale == 1 (bitwise copy / cast).
+ *  src, dst    device, 16-byte aligned; may be the same pointer only when
+ *              src_dtype == dst_dtype (in place).  FLKL_DTYPE_F32 or
+ *              FLKL_DTYPE_BF16 each (bf16 results rounded to nearest even).
+ *  scale       device fp32 scalar read on the device (no host
+ *              synchronisation), or NULL for 1.
+ *  Asynchronous on `stream`.  n < 0, a bad dtype or a null src/dst with
+ *  n > 0 gives FLKL_ERR_INVALID_ARG; misaligned pointers
+ *  FLKL_ERR_UNSUPPORTED. */
+FLKL_API flkl_status flkl_scale_cast(const void* src, int src_dtype, void* dst, int dst_dtype,
+                                     int64_t n, const float* scale, void* stream);
+
 /* Kinds of launches reported by flkl_forward_backward_profiled. */
 typedef enum {
   FLKL_LAUNCH_PREPARE = 0,  /* valid-row count and divisor                   */
@@ -288,9 +304,10 @@ FLKL_API flkl_status flkl_forward_backward_profiled(
  *  - Sizes whose flkl_workspace_size() exceeds FLKL_NOALLOC_SCRATCH_BYTES
  *    return FLKL_ERR_TOO_LARGE before any launch (BT=1024, H=4096,
  *    V=128256 with dW needs 98.6 MiB and fits).
- *  - The first call on a device looks up the scratch address on that device
- *    (the device must be current); make that first call before any stream
- *    capture.
+ *  - Every call looks up the scratch address on the current device (a
+ *    host-side lookup, so a device reset cannot leave a stale address); the
+ *    first call on a device also loads the library's device code there, so
+ *    make that first call before any stream capture.
  *  - Every call on a device shares the one scratch array, which keeps the
  *    previous call's contents (the call initialises what it reads).  Calls
  *    that can overlap on the GPU (different streams, or different host

@@ -26,7 +26,7 @@ __all__ = [
     "flkl_ce_forward_backward_dp", "count_valid", "flkl_selective_logprob_forward",
     "flkl_selective_logprob_backward", "selective_logprob", "SelectiveLogProb",
     "flkl_jsd_workspace_size", "flkl_jsd_forward_backward", "jsd_forward_backward",
-    "FusedLinearJSDLoss",
+    "FusedLinearJSDLoss", "flkl_scale_cast",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -108,6 +108,9 @@ def _lib():
             c.c_int64, c.c_int64, c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_float,
             c.c_float, c.c_int, c.c_int, c.c_int, c.c_int, c.c_void_p, c.c_void_p, c.c_void_p,
             c.c_void_p, c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.flkl_scale_cast.restype = c.c_int
+        lib.flkl_scale_cast.argtypes = [c.c_void_p, c.c_int, c.c_void_p, c.c_int, c.c_int64,
+                                        c.c_void_p, c.c_void_p]
         lib.flkl_count_valid.restype = c.c_int
         lib.flkl_count_valid.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p]
         lib.flkl_forward_backward_noalloc.restype = c.c_int
@@ -306,6 +309,11 @@ def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H
     return st, [kinds[i] for i in range(k)], [flops[i] for i in range(k)], n.value
 
 
+def flkl_scale_cast(src, src_dtype, dst, dst_dtype, n, scale, stream=None) -> int:
+    return _lib().flkl_scale_cast(src, int(src_dtype), dst, int(dst_dtype), int(n), scale,
+                                  stream)
+
+
 def flkl_device_status(workspace_ptr, stream=None) -> int:
     return _lib().flkl_device_status(workspace_ptr, stream)
 
@@ -333,6 +341,58 @@ def _check_dev(name, t, dtype, shape, device):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _outputs(out: Optional[dict], dev, BT: int, H: int, V: int, dt, pdt, compute_dW: bool,
+             compute_db: bool) -> tuple:
+    """loss, dX, dW, db for one call: each caller-supplied tensor of ``out``
+    is checked against the shape, dtype and device this call writes (the
+    kernels write BT*H, V*H and V elements, so a smaller buffer would be
+    written past its end); missing ones are allocated."""
+    out = {} if out is None else out
+    specs = {"loss": (torch.float32, ()), "dX": (dt, (BT, H)),
+             "dW": (pdt, (V, H)) if compute_dW else None,
+             "db": (pdt, (V,)) if compute_db else None}
+    res = []
+    for name, spec in specs.items():
+        if spec is None:
+            res.append(None)
+            continue
+        t = out.get(name)
+        if t is None:
+            t = torch.empty(spec[1], dtype=spec[0], device=dev)
+        else:
+            _check_dev(f"out[{name!r}]", t, spec[0], spec[1], dev)
+        res.append(t)
+    return tuple(res)
+
+
+def _workspace(workspace: Optional[torch.Tensor], need: int, dev) -> torch.Tensor:
+    """The caller's workspace when it is a large enough contiguous uint8
+    buffer on ``dev``, else a new one."""
+    if workspace is not None:
+        if workspace.device != dev or workspace.dtype != torch.uint8 or \
+                not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous uint8 tensor on " + str(dev))
+        if workspace.numel() >= need:
+            return workspace
+    return torch.empty(need, dtype=torch.uint8, device=dev)
+
+
+def _scaled(t: Optional[torch.Tensor], grad_out: torch.Tensor, dtype) -> Optional[torch.Tensor]:
+    """``t * grad_out`` in ``dtype`` as a new tensor, by the CUDA library:
+    the incoming gradient is read on the device (no host synchronisation)
+    and the product is skipped when it is 1."""
+    if t is None:
+        return None
+    out = torch.empty(t.shape, dtype=dtype, device=t.device)
+    g = grad_out.detach().to(device=t.device, dtype=torch.float32).reshape(()).contiguous()
+    st = torch.cuda.current_stream(t.device)
+    s = flkl_scale_cast(_ptr(t), DTYPES[t.dtype], _ptr(out), DTYPES[dtype], t.numel(), _ptr(g),
+                        st.cuda_stream)
+    if s != FLKL_OK:
+        raise FlklError(s, "flkl_scale_cast")
+    return out
 
 
 def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor], Q: torch.Tensor,
@@ -367,24 +427,11 @@ def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
         _check_dev("shift_labels", shift_labels, torch.int64, (BT,), dev)
     compute_db = bool(compute_db and b is not None)
     pdt = torch.float32 if (accum_fp32 or dt == torch.float32) else dt
-    out = {} if out is None else out
-    loss = out.get("loss")
-    if loss is None:
-        loss = torch.empty((), dtype=torch.float32, device=dev)
-    dX = out.get("dX")
-    if dX is None:
-        dX = torch.empty_like(X)
-    dW = out.get("dW") if compute_dW else None
-    if compute_dW and dW is None:
-        dW = torch.empty((V, H), dtype=pdt, device=dev)
-    db = out.get("db") if compute_db else None
-    if compute_db and db is None:
-        db = torch.empty((V,), dtype=pdt, device=dev)
+    loss, dX, dW, db = _outputs(out, dev, BT, H, V, dt, pdt, compute_dW, compute_db)
     need = flkl_workspace_size(BT, H, V, DTYPES[dt], compute_dW, compute_db)
     if need == 0:
         raise FlklError(1, "flkl_workspace_size")
-    if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    workspace = _workspace(workspace, need, dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
     args = (_ptr(X), _ptr(W), _ptr(b), _ptr(Q), _ptr(shift_labels), ignore_index, BT, H, V,
             DTYPES[dt], temperature, eps, REDUCTIONS[reduction], compute_dW, compute_db,
@@ -424,15 +471,11 @@ class _FusedLinearKLDivFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, grad_out):
         dX, dW, db = ctx.saved_tensors
-        one = bool((grad_out == 1).all())
-        if not one:
-            dX = dX * grad_out.to(dX.dtype)
-            dW = None if dW is None else dW * grad_out.to(dW.dtype)
-            db = None if db is None else db * grad_out.to(db.dtype)
-        if dW is not None:
-            dW = dW.to(ctx.w_dtype)
-        if db is not None:
-            db = db.to(ctx.w_dtype)
+        # one pass each: scale by the incoming gradient and cast to the
+        # parameter dtype, on the device
+        dX = _scaled(dX, grad_out, dX.dtype)
+        dW = _scaled(dW, grad_out, ctx.w_dtype)
+        db = _scaled(db, grad_out, ctx.w_dtype)
         return dX, dW, db, None, None, None, None, None, None, None
 
 
@@ -493,24 +536,11 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
         _check_dev("b", b, dt, (V,), dev)
     compute_db = bool(compute_db and b is not None)
     pdt = torch.float32 if (accum_fp32 or dt == torch.float32) else dt
-    out = {} if out is None else out
-    loss = out.get("loss")
-    if loss is None:
-        loss = torch.empty((), dtype=torch.float32, device=dev)
-    dX = out.get("dX")
-    if dX is None:
-        dX = torch.empty_like(X)
-    dW = out.get("dW") if compute_dW else None
-    if compute_dW and dW is None:
-        dW = torch.empty((V, H), dtype=pdt, device=dev)
-    db = out.get("db") if compute_db else None
-    if compute_db and db is None:
-        db = torch.empty((V,), dtype=pdt, device=dev)
+    loss, dX, dW, db = _outputs(out, dev, BT, H, V, dt, pdt, compute_dW, compute_db)
     need = flkl_workspace_size(BT, H, V, DTYPES[dt], compute_dW, compute_db)
     if need == 0:
         raise FlklError(1, "flkl_workspace_size")
-    if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    workspace = _workspace(workspace, need, dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
     args = (_ptr(X), _ptr(W), _ptr(b), _ptr(target), ignore_index, BT, H, V, DTYPES[dt],
             temperature, REDUCTIONS[reduction], compute_dW, compute_db, accum_fp32, _ptr(loss),
@@ -569,8 +599,7 @@ def jsd_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Ten
     need = flkl_jsd_workspace_size(BT, H, Ht, V, DTYPES[dt], compute_dW, compute_db)
     if need == 0:
         raise FlklError(1, "flkl_jsd_workspace_size")
-    if workspace is None or workspace.numel() < need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    workspace = _workspace(workspace, need, dev)
     st = stream if stream is not None else torch.cuda.current_stream(dev)
     status = flkl_jsd_forward_backward(
         _ptr(X), _ptr(W), _ptr(b), _ptr(Xt), _ptr(Wt), _ptr(bt), _ptr(shift_labels),
@@ -603,14 +632,11 @@ class _FusedLinearJSDFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, grad_out):
         dX, dW, db = ctx.saved_tensors
-        if not bool((grad_out == 1).all()):
-            dX = dX * grad_out.to(dX.dtype)
-            dW = None if dW is None else dW * grad_out.to(dW.dtype)
-            db = None if db is None else db * grad_out.to(db.dtype)
-        if dW is not None:
-            dW = dW.to(ctx.w_dtype)
-        if db is not None:
-            db = db.to(ctx.w_dtype)
+        # one pass each: scale by the incoming gradient and cast to the
+        # parameter dtype, on the device
+        dX = _scaled(dX, grad_out, dX.dtype)
+        dW = _scaled(dW, grad_out, ctx.w_dtype)
+        db = _scaled(db, grad_out, ctx.w_dtype)
         return dX, dW, db, None, None, None, None, None, None, None, None, None
 
 
@@ -766,14 +792,11 @@ class _FusedLinearCEFunction(torch.autograd.Function):
     @staticmethod
     def backward(ctx, grad_out):
         dX, dW, db = ctx.saved_tensors
-        if not bool((grad_out == 1).all()):
-            dX = dX * grad_out.to(dX.dtype)
-            dW = None if dW is None else dW * grad_out.to(dW.dtype)
-            db = None if db is None else db * grad_out.to(db.dtype)
-        if dW is not None:
-            dW = dW.to(ctx.w_dtype)
-        if db is not None:
-            db = db.to(ctx.w_dtype)
+        # one pass each: scale by the incoming gradient and cast to the
+        # parameter dtype, on the device
+        dX = _scaled(dX, grad_out, dX.dtype)
+        dW = _scaled(dW, grad_out, ctx.w_dtype)
+        db = _scaled(db, grad_out, ctx.w_dtype)
         return dX, dW, db, None, None, None, None, None
 
 

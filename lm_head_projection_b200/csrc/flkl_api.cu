@@ -980,24 +980,23 @@ flkl_status jsd_impl(const void* X, const void* W, const void* b, const void* Xt
 // library, without any allocation call.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FLKL_NOALLOC_SCRATCH_BYTES];
 
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the fixed scratch on the current device, looked up once
-// per device.  In host code the symbol is only a host-side handle: the
-// address a kernel may use comes from cudaGetSymbolAddress.
+// Device address of the fixed scratch on the current device.  In host code
+// the symbol is only a host-side handle: the address a kernel may use comes
+// from cudaGetSymbolAddress.  It is looked up on every call (a host-side
+// lookup once the library's device code is loaded on the device), so that a
+// device reset, which reloads the device code at a possibly different
+// address, never leaves a stale address behind.  The first call on a device
+// loads the device code there.
 cudaError_t noalloc_scratch(void** out) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);  // a device must be current
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  (void)dev;
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  if (p == nullptr) return cudaErrorInvalidSymbol;
+  *out = p;
   return cudaSuccess;
 }
 
@@ -1051,6 +1050,36 @@ flkl_status flkl_ce_forward_backward(const void* X, const void* W, const void* b
                                temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
                                BT > 0 ? target : nullptr);
+}
+
+flkl_status flkl_scale_cast(const void* src, int src_dtype, void* dst, int dst_dtype,
+                            int64_t n, const float* scale, void* stream) {
+  const bool ok_dt = (src_dtype == FLKL_DTYPE_F32 || src_dtype == FLKL_DTYPE_BF16) &&
+                     (dst_dtype == FLKL_DTYPE_F32 || dst_dtype == FLKL_DTYPE_BF16);
+  if (n < 0 || !ok_dt) return FLKL_ERR_INVALID_ARG;
+  if (n == 0) return FLKL_OK;
+  if (src == nullptr || dst == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (src == dst && src_dtype != dst_dtype) return FLKL_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(scale) & 3u))
+    return FLKL_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long vecs = std::max<long long>(1, n / 8);
+  const unsigned grid = static_cast<unsigned>(
+      std::min<long long>(cdiv(vecs, 256), static_cast<long long>(num_sms()) * 8));
+  const bool sf = src_dtype == FLKL_DTYPE_F32, df = dst_dtype == FLKL_DTYPE_F32;
+  if (sf && df)
+    k_scale_cast<float, float><<<grid, 256, 0, st>>>(static_cast<const float*>(src),
+                                                     static_cast<float*>(dst), n, scale);
+  else if (sf)
+    k_scale_cast<float, __nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const float*>(src), static_cast<__nv_bfloat16*>(dst), n, scale);
+  else if (df)
+    k_scale_cast<__nv_bfloat16, float><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(src), static_cast<float*>(dst), n, scale);
+  else
+    k_scale_cast<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), n, scale);
+  return cudaGetLastError() == cudaSuccess ? FLKL_OK : FLKL_ERR_CUDA;
 }
 
 flkl_status flkl_count_valid(const int64_t* labels, int64_t BT, int64_t ignore_index,

@@ -198,4 +198,59 @@ __global__ void k_zero(void* p, size_t bytes) {
     for (size_t j = i; j < bytes; ++j) static_cast<uint8_t*>(p)[j] = 0;
 }
 
+// dst = cast(src * s) over n elements, s = *scale (1 when scale is NULL; the
+// product is skipped when s == 1).  Grid-stride over 8-element vectors, then
+// a scalar tail; src and dst 16-byte aligned, possibly the same buffer (each
+// element is read and written by the same thread).
+template <class TS>
+__device__ __forceinline__ float ld_as_f32(const TS* p, size_t i) {
+  if constexpr (sizeof(TS) == 4) return p[i];
+  else return __bfloat162float(p[i]);
+}
+template <class TD>
+__device__ __forceinline__ void st_from_f32(TD* p, size_t i, float v) {
+  if constexpr (sizeof(TD) == 4) p[i] = v;
+  else p[i] = __float2bfloat16_rn(v);
+}
+template <class TS, class TD>
+__global__ void __launch_bounds__(256) k_scale_cast(const TS* src, TD* dst, long long n,
+                                                    const float* scale) {
+  const float s = scale != nullptr ? *scale : 1.f;
+  const bool mul = s != 1.f;
+  const long long nv = n / 8;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < nv;
+       v += stride) {
+    float f[8];
+    if constexpr (sizeof(TS) == 4) {
+      const float4 a = reinterpret_cast<const float4*>(src)[2 * v];
+      const float4 b = reinterpret_cast<const float4*>(src)[2 * v + 1];
+      f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+      f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    } else {
+      unpack8_bf16(reinterpret_cast<const uint4*>(src)[v], f);
+    }
+    if (mul) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) f[j] *= s;
+    }
+    if constexpr (sizeof(TD) == 4) {
+      reinterpret_cast<float4*>(dst)[2 * v] = make_float4(f[0], f[1], f[2], f[3]);
+      reinterpret_cast<float4*>(dst)[2 * v + 1] = make_float4(f[4], f[5], f[6], f[7]);
+    } else {
+      uint4 u;
+      u.x = pack_bf16x2(f[0], f[1]);
+      u.y = pack_bf16x2(f[2], f[3]);
+      u.z = pack_bf16x2(f[4], f[5]);
+      u.w = pack_bf16x2(f[6], f[7]);
+      reinterpret_cast<uint4*>(dst)[v] = u;
+    }
+  }
+  for (long long i = nv * 8 + blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+       i < n; i += stride) {
+    const float x = ld_as_f32<TS>(src, static_cast<size_t>(i));
+    st_from_f32<TD>(dst, static_cast<size_t>(i), mul ? x * s : x);
+  }
+}
+
 }  // namespace flkl

@@ -34,7 +34,9 @@ class DataParallelFusedLinearLoss:
     or "ce" (integer targets [BT], which are also the row mask).  Options are
     those of :func:`forward_backward` / :func:`cross_entropy_forward_backward`.
     ``group`` is the process group (default: the world).  Outputs are reused
-    from step to step (``out`` and the workspace stay allocated).
+    from step to step while the shapes and flags stay the same (``out`` and
+    the workspace stay allocated), so a step's results are overwritten by
+    the next step's.
     """
 
     def __init__(self, kind: str = "kl", group=None, ignore_index: int = -100,
@@ -52,9 +54,22 @@ class DataParallelFusedLinearLoss:
     def _count(self, mask_labels: Optional[torch.Tensor], BT: int, device) -> torch.Tensor:
         return count_valid(mask_labels, BT, self.ignore_index, device=device)
 
+    def _reusable_out(self, X, W, b, compute_dW, compute_db) -> Optional[dict]:
+        """The previous step's outputs when this step writes the same shapes,
+        dtypes and gradients (else None, and the call allocates new ones): a
+        short last batch, or a change of the flags, must not reuse buffers
+        sized for another step."""
+        key = (tuple(X.shape), tuple(W.shape), X.dtype, X.device, bool(compute_dW),
+               bool(compute_db and b is not None), bool(self.accum_fp32))
+        if key != getattr(self, "_out_key", None):
+            self.out = None
+            self._out_key = key
+        return self.out
+
     def _local(self, X, W, b, teacher, labels, n_total, compute_dW, compute_db) -> dict:
+        out = self._reusable_out(X, W, b, compute_dW, compute_db)
         common = dict(compute_dW=compute_dW, compute_db=compute_db, accum_fp32=self.accum_fp32,
-                      out=self.out, workspace=self.workspace, n_valid_total=n_total)
+                      out=out, workspace=self.workspace, n_valid_total=n_total)
         if self.kind == "ce":
             r = cross_entropy_forward_backward(X, W, b, teacher, self.ignore_index,
                                                self.temperature, self.reduction, **common)

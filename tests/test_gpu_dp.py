@@ -111,3 +111,43 @@ def test_one_rank_nccl_group_gives_the_direct_call(kind):
         dist.destroy_process_group()
     for k in ("loss", "dX", "dW", "db"):
         assert torch.equal(r[k], direct[k]), k
+
+
+def test_steps_of_changing_batch_size_get_buffers_of_their_own_size():
+    """A data-parallel loss object reused over steps of 96, 64 and 128 rows
+    (a short batch, then a longer one) gives every step the direct call's
+    bytes: outputs sized for another step are never reused."""
+    import torch.distributed as dist
+
+    import lm_head_projection_b200 as pkg
+    from lm_head_projection_b200.dp import DataParallelFusedLinearLoss
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda:0"))
+    try:
+        loss = DataParallelFusedLinearLoss("kl", temperature=1.5)
+        for i, (BT, flags) in enumerate([(96, (True, True)), (64, (True, True)),
+                                         (128, (True, True)), (128, (False, True)),
+                                         (128, (True, False))]):
+            w = small_case(dtype="bf16", BT=BT, H=128, V=1000, bias=True, ignore_frac=0.1,
+                           temperature=1.5, seed=30 + i)
+            g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v)
+                 for k, v in make_inputs(w).items()}
+            cw, cb = flags
+            r = loss.step(g["X"], g["W"], g["b"], g["Q"], g["shift_labels"], compute_dW=cw,
+                          compute_db=cb)
+            direct = pkg.forward_backward(g["X"], g["W"], g["b"], g["Q"], g["shift_labels"],
+                                          g["ignore_index"], g["temperature"], g["eps"],
+                                          g["reduction"], compute_dW=cw, compute_db=cb,
+                                          accum_fp32=True, check_status=True)
+            torch.cuda.synchronize()
+            assert r["dX"].shape == (BT, 128)
+            for k in ("loss", "dX", "dW", "db"):
+                if direct[k] is None:
+                    assert r[k] is None, k
+                else:
+                    assert torch.equal(r[k], direct[k]), (BT, k)
+    finally:
+        dist.destroy_process_group()

@@ -8,7 +8,11 @@ every device.  These tests call it through the C ABI and check that it gives
 what the workspace entry point gives, within the parity tolerances, on two
 calls in a row (the scratch keeps the previous call's contents, which must
 not leak into the next result), and that sizes beyond the scratch are
-refused before anything runs.  This file is collected last.
+refused before anything runs.  Both entry points run the same deterministic
+kernels on the same bytes, so the results are also compared bitwise; a
+sequence of different plans (a large one, then smaller ones of other dtypes
+and flags, then the large one again) shows that no stale scratch contents
+reach a result.  This file is collected last.
 """
 
 import numpy as np
@@ -68,6 +72,44 @@ def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(w):
         assert _call_noalloc(g, w, out) == 0
         torch.cuda.synchronize()
         _close(w.dtype, out, ref)
+        _same_bytes(out, ref)
+
+
+def _same_bytes(got, ref):
+    for k in ("loss", "dX", "dW", "db"):
+        if ref[k] is None:
+            assert got[k] is None, k
+        else:
+            assert torch.equal(got[k], ref[k]), k
+
+
+# A large plan first (most of the scratch: a 1024-row, 16384-column head with
+# dW), then smaller ones with other dtypes and flags, then the large one again.
+SEQUENCE = [
+    small_case(dtype="bf16", BT=1024, H=4096, V=16384, bias=False, reduction="batchmean",
+               w_std=0.02, seed=21),
+    small_case(dtype="bf16", BT=77, H=128, V=1032, bias=True, reduction="mean",
+               ignore_frac=0.2, zero_frac=0.05, temperature=1.5, seed=22),
+    small_case(dtype="fp32", BT=50, H=64, V=520, bias=True, reduction="sum", seed=23),
+    small_case(dtype="bf16", BT=300, H=256, V=4104, bias=True, reduction="batchmean",
+               compute_dW=False, seed=24),
+]
+
+
+def test_noalloc_interleaved_plans_give_the_workspace_entry_bytes():
+    dev = torch.device("cuda:0")
+    runs = []
+    for w in SEQUENCE:
+        inp = make_inputs(w)
+        runs.append((w, {k: (v.to(dev) if isinstance(v, torch.Tensor) else v)
+                         for k, v in inp.items()}, run_gpu(inp)))
+    for w, g, ref in runs + runs[:1]:
+        out = {k: (None if ref[k] is None else torch.full_like(ref[k], float("nan")))
+               for k in ("loss", "dX", "dW", "db")}
+        assert _call_noalloc(g, w, out) == 0
+        torch.cuda.synchronize()
+        _close(w.dtype, out, ref)
+        _same_bytes(out, ref)
 
 
 def test_noalloc_refuses_sizes_beyond_the_scratch():
