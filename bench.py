@@ -112,6 +112,12 @@ def parse():
     ap.add_argument("--norm-shape", default="8192x8192", help="ROWSxH for --op *_norm")
     ap.add_argument("--norm-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--frozen", action="store_true", help="norm weight (and bias) frozen")
+    ap.add_argument("--calls", type=int, default=0,
+                    help="profiling helper: run this many plain calls of --workload through "
+                         "the public API, print their CUDA-event times and exit (no bench "
+                         "line); a small case for ncu is --workload NAME with --rows R")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="with --calls: take the workload with BT=R rows instead of its own")
     ap.add_argument("--dp", action="store_true",
                     help="data-parallel training step: whole-batch kept-row count and "
                          "all-reduce of loss, dW, db (NCCL) inside each timed step")
@@ -779,9 +785,49 @@ def run_jsd(args):
     print(json.dumps(line), flush=True)
 
 
+def run_calls(args):
+    """A few plain calls of one workload (for profilers such as ncu): inputs
+    drawn on the device, each call timed with CUDA events, device status
+    checked at the end."""
+    import lm_head_projection_b200 as pkg
+
+    w = ALL_WORKLOADS[args.workload]
+    if args.rows:
+        w = w.with_(BT=args.rows)
+    dev = torch.device("cuda", 0)
+    inp = make_inputs(w, device=dev)
+    r, times = None, []
+    for _ in range(args.calls):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        if w.ce:
+            r = pkg.cross_entropy_forward_backward(
+                inp["X"], inp["W"], inp["b"], inp["target"], inp["ignore_index"],
+                inp["temperature"], inp["reduction"], compute_dW=inp["compute_dW"],
+                compute_db=inp["compute_db"], accum_fp32=inp["accum_fp32"], out=r,
+                workspace=None if r is None else r["workspace"])
+        else:
+            r = pkg.forward_backward(inp["X"], inp["W"], inp["b"], inp["Q"], inp["shift_labels"],
+                                     inp["ignore_index"], inp["temperature"], inp["eps"],
+                                     inp["reduction"], compute_dW=inp["compute_dW"],
+                                     compute_db=inp["compute_db"], accum_fp32=inp["accum_fp32"],
+                                     out=r, workspace=None if r is None else r["workspace"])
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(round(e0.elapsed_time(e1), 4))
+    status = pkg.flkl_device_status(r["workspace"].data_ptr(),
+                                    torch.cuda.current_stream().cuda_stream) if r else 0
+    print(json.dumps({"workload": w.name, "BT": w.BT, "H": w.H, "V": w.V, "ms": times,
+                      "status": status}), flush=True)
+    if status != 0:
+        raise SystemExit(1)
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.op == "jsd":
+    if a.calls > 0:
+        run_calls(a)
+    elif a.op == "jsd":
         run_jsd(a)
     elif a.op == "logprob":
         run_logprob(a)

@@ -35,9 +35,17 @@ namespace flkl {
 constexpr int TC_BM = 256;            // output tile rows (pair)
 constexpr int TC_BN = 256;            // output tile columns
 constexpr int TC_HM = 128;            // rows per CTA
-constexpr int TC_BK = 128;            // K depth of a ring stage (a multiple of 64)
+// Build-time tunables (-DFLKL_TC_BK=..., -DFLKL_TC_STAGES=...).
+#ifndef FLKL_TC_BK
+#define FLKL_TC_BK 128
+#endif
+#ifndef FLKL_TC_STAGES
+#define FLKL_TC_STAGES 3
+#endif
+constexpr int TC_BK = FLKL_TC_BK;     // K depth of a ring stage (a multiple of 64)
 constexpr int TC_KSUB = TC_BK / 64;   // 128-byte swizzle atoms along K per stage
-constexpr int TC_STAGES = 3;
+constexpr int TC_STAGES = FLKL_TC_STAGES;
+static_assert(TC_BK % 64 == 0 && TC_BK <= 256, "stage depth: a multiple of 64, at most 256");
 constexpr int TC_PREFETCH_KB = 0;     // L2 prefetch distance of the producer, in k-blocks
 constexpr int TC_EPI_WARPS = 8;       // two per TMEM lane quarter
 constexpr int TC_EPI_COLS = 128;      // accumulator columns per epilogue warp

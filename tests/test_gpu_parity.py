@@ -189,13 +189,24 @@ def _sample(n, k, seed):
     return sorted(rows)
 
 
+def _tile_edges(n, tile=256):
+    """First and last index of every `tile`-wide block of [0, n): every
+    vocabulary chunk of the CUDA path starts and ends on such a block, so
+    these rows include each chunk's first and last row (the ragged last
+    chunk among them), whatever the chunk width."""
+    rows = set()
+    for t0 in range(0, n, tile):
+        rows |= {t0, min(n, t0 + tile) - 1}
+    return rows
+
+
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_full_size_workload(name):
     w = WORKLOADS[name]
     inp = make_inputs(w)
     got = run_gpu(inp)
     dx_rows = _sample(w.BT, 24, 1)
-    dw_rows = _sample(w.V, 24, 2) if w.compute_dW else None
+    dw_rows = sorted(set(_sample(w.V, 24, 2)) | _tile_edges(w.V)) if w.compute_dW else None
     ref = run_oracle(inp, dX_rows=dx_rows, dW_rows=dw_rows)
     assert_close(w.dtype, got, ref, dX_rows=dx_rows, dW_rows=dw_rows)
     # dX rows of dropped rows are exactly zero
