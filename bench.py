@@ -103,12 +103,15 @@ def parse():
     ap.add_argument("--cpu-sample-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip timing the other bf16 workloads after the headline")
     ap.add_argument("--op", default="loss",
-                    choices=["loss", "rms_norm", "layer_norm", "logprob", "jsd"],
+                    choices=["loss", "rms_norm", "layer_norm", "logprob", "jsd", "memory"],
                     help="loss: the fused linear KL / CE loss (default); rms_norm / "
                          "layer_norm: the norm backward with frozen-parameter flags; logprob: "
                          "selective log-probability forward + backward on a CE workload; "
-                         "jsd: fused linear JSD with a teacher head of the same shape")
+                         "jsd: fused linear JSD with a teacher head of the same shape; "
+                         "memory: peak device memory of one call at the pages' head shape")
     ap.add_argument("--norm-shape", default="8192x8192", help="ROWSxH for --op *_norm")
     ap.add_argument("--norm-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--frozen", action="store_true", help="norm weight (and bias) frozen")
@@ -127,24 +130,35 @@ def parse():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons every 20 ms in the background;
+    summary() keeps the samples taken between mark_start() and mark_end()
+    (the timed region), by nvidia-smi's own timestamps."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.path = tempfile.mktemp(prefix="flkl_clocks_", suffix=".csv")
         self.proc = None
-        self.t_start = time.time()
+        self.t0 = self.t1 = None
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "-lms", "20", "-i", str(gpu_index)], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def stop(self):
         if self.proc is not None:
+            time.sleep(0.05)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -155,27 +169,35 @@ class ClockSampler:
     def summary(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        import datetime
+
         rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[3], parts[4:]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[4], parts[5:]))
                 except ValueError:
                     continue
         os.unlink(self.path)
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        inside = [r for r in rows if self.t0 is not None and self.t1 is not None
+                  and self.t0 <= r[0] <= self.t1]
+        window = "timed region"
+        if not inside:  # a region shorter than the sampling period: the nearest sample after it
+            after = [r for r in rows if self.t1 is not None and r[0] >= self.t1]
+            inside, window = (after[:1] or rows[-1:]), "first sample after the timed region"
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        # samples under load: the upper half of the observed clocks
-        clocks = sorted(r[0] for r in rows)
-        active = [r for r in rows if r[0] >= clocks[len(clocks) // 4]]
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3][1:5])
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[4][1:5])
                           if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in active), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+        power = [float(r[3]) for r in inside if r[3].replace(".", "", 1).isdigit()]
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": rows[0][2],
+                "reasons": reasons, "samples": len(inside), "window": window,
+                "power_w_median": statistics.median(power) if power else None}
 
 
 # ------------------------------------------------------------------ helpers
@@ -246,6 +268,193 @@ def time_oracle(args, kw):
 
 # ------------------------------------------------------------------ our arm
 
+class Case:
+    """One workload's inputs, outputs and the raw C-ABI arguments of its call
+    (the public API is called once to allocate outputs and the workspace)."""
+
+    def __init__(self, pkg, w, dev, stream):
+        self.pkg, self.w, self.stream = pkg, w, stream
+        inp = make_inputs(w, device=dev)
+        self.inp = inp
+        X, W, b, Q, lab = inp["X"], inp["W"], inp["b"], inp["Q"], inp["shift_labels"]
+        tgt = inp.get("target")
+        self.compute_db = inp["compute_db"]
+        r0 = self.api_call(check_status=True)
+        self.ws = r0["workspace"]
+        self.out = {k: r0[k] for k in ("loss", "dX", "dW", "db")}
+        p = lambda t: None if t is None else t.data_ptr()
+        dt_code = pkg.DTYPES[X.dtype]
+        out, ws = self.out, self.ws
+        self.kl_args = (p(X), p(W), p(b), p(Q), p(lab), inp["ignore_index"], w.BT, w.H, w.V,
+                        dt_code, inp["temperature"], inp["eps"],
+                        pkg.REDUCTIONS[inp["reduction"]], inp["compute_dW"], self.compute_db,
+                        inp["accum_fp32"], p(out["loss"]), p(out["dX"]), p(out["dW"]),
+                        p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
+        self.ce_args = (p(X), p(W), p(b), p(tgt), inp["ignore_index"], w.BT, w.H, w.V, dt_code,
+                        inp["temperature"], pkg.REDUCTIONS[inp["reduction"]],
+                        inp["compute_dW"], self.compute_db, inp["accum_fp32"], p(out["loss"]),
+                        p(out["dX"]), p(out["dW"]), p(out["db"]), p(ws), ws.numel(),
+                        stream.cuda_stream)
+        self.tgt_ptr = p(tgt)
+
+    def api_call(self, out=None, workspace=None, check_status=False):
+        """The public Python API call a user makes for this workload."""
+        pkg, w, inp = self.pkg, self.w, self.inp
+        if w.ce:
+            return pkg.cross_entropy_forward_backward(
+                inp["X"], inp["W"], inp["b"], inp["target"], inp["ignore_index"],
+                inp["temperature"], inp["reduction"], compute_dW=inp["compute_dW"],
+                compute_db=self.compute_db, accum_fp32=inp["accum_fp32"], out=out,
+                workspace=workspace, check_status=check_status)
+        return pkg.forward_backward(inp["X"], inp["W"], inp["b"], inp["Q"], inp["shift_labels"],
+                                    inp["ignore_index"], inp["temperature"], inp["eps"],
+                                    inp["reduction"], compute_dW=inp["compute_dW"],
+                                    compute_db=self.compute_db, accum_fp32=inp["accum_fp32"],
+                                    out=out, workspace=workspace, check_status=check_status)
+
+    def call(self) -> int:
+        pkg = self.pkg
+        return (pkg.flkl_ce_forward_backward(*self.ce_args) if self.w.ce
+                else pkg.flkl_forward_backward(*self.kl_args))
+
+    def profiled_steps(self, steps: int, cap: int = 32):
+        """`steps` calls through the profiled entry, events around every
+        launch, no synchronisation between calls (the same back-to-back launch
+        stream as the timed steps).  Returns per-kind [ms, launches, GEMM
+        FLOPs], the launches per call, and the elapsed ms per call from the
+        first event to the last."""
+        pkg, st = self.pkg, self.stream
+        events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap * steps)]
+        for e in events:  # torch creates the CUDA event on its first record
+            e.record(st)
+        torch.cuda.synchronize()
+        recs = []
+        for i in range(steps):
+            r = pkg.flkl_forward_backward_profiled(*self.kl_args,
+                                                   events[2 * cap * i: 2 * cap * (i + 1)], cap,
+                                                   ce_target=self.tgt_ptr)
+            if r[0] != 0:
+                raise pkg.FlklError(r[0], "flkl_forward_backward_profiled")
+            if r[3] > cap:
+                raise RuntimeError(f"{r[3]} launches per call exceed the {cap} recorded")
+            recs.append(r)
+        torch.cuda.synchronize()
+        per_kind = {}
+        for i, (_, kinds, flops, n) in enumerate(recs):
+            base = 2 * cap * i
+            for j, k in enumerate(kinds):
+                d = per_kind.setdefault(pkg.LAUNCH_KINDS[k], [0.0, 0, 0.0])
+                d[0] += events[base + 2 * j].elapsed_time(events[base + 2 * j + 1])
+                d[1] += 1
+                d[2] += flops[j]
+        n = recs[0][3]
+        elapsed = events[0].elapsed_time(events[2 * cap * (steps - 1) + 2 * n - 1])
+        return per_kind, n, elapsed / steps
+
+
+def sm_clock_summary(buf: torch.Tensor, window_ms: float):
+    """Median, 10th and 90th percentile SM clock (MHz) of a flkl_clock_trace
+    record over its first `window_ms`."""
+    a = buf.cpu().tolist()
+    t, c = a[0::2], a[1::2]
+    mhz = []
+    for i in range(1, len(t)):
+        if t[i] - t[0] > window_ms * 1e6:
+            break
+        if t[i] > t[i - 1]:
+            mhz.append((c[i] - c[i - 1]) / (t[i] - t[i - 1]) * 1e3)
+    if not mhz:
+        return None
+    mhz.sort()
+    return {"median": round(statistics.median(mhz)), "p10": round(mhz[len(mhz) // 10]),
+            "p90": round(mhz[(9 * len(mhz)) // 10]), "samples": len(mhz)}
+
+
+def timed_steps(case, steps, barrier=lambda: None):
+    """Exactly `steps` calls between two events on the launch stream, with a
+    barrier and a synchronisation on both sides; returns elapsed ms."""
+    st = case.stream
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        s = case.call()
+        if s != 0:
+            raise case.pkg.FlklError(s, "flkl_forward_backward")
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1)
+
+
+def kernel_roofline(w, per_kind, steps, peaks, peaks_src, ms_per_step):
+    """Roofline of the dominant kernel, tc_group_kernel (every GEMM launch of
+    a step: pass 1, pass 2 of the first chunk and one grouped launch per
+    vocabulary chunk), over a step: the method's counted FLOPs (one logits
+    GEMM, dX and dW when trained: 2*BT*H*V each) per step over the kernel's
+    device time per step, against the measured burst bf16 peak (the timed
+    region is a few hundred ms at most); the executed FLOPs (adding the
+    recompute of the logits in pass 2) are reported beside it."""
+    gemm_kinds = [k for k, v in per_kind.items() if v[2] > 0]
+    gemm_ms = sum(per_kind[k][0] for k in gemm_kinds) / steps
+    launches = sum(per_kind[k][1] for k in gemm_kinds) / steps
+    executed = sum(per_kind[k][2] for k in gemm_kinds) / steps
+    counted = w.flops_counted()
+    burst = peaks["bf16_tflops"]
+    sust = peaks.get("bf16_tflops_sustained", burst)
+    achieved = counted / (gemm_ms * 1e-3) / 1e12
+    traffic = None
+    parts = {k: dram_traffic(w.name, k) for k in gemm_kinds}
+    if all(v is not None for v in parts.values()) and parts:
+        traffic = sum(parts[k] * per_kind[k][1] / steps for k in gemm_kinds)
+    algo = algorithmic_bytes(w)
+    kind_name = "tc_group_kernel" if w.dtype == "bf16" else "k_simt_* (fp32 FMA)"
+    return {
+        "bound": "tensor" if w.dtype == "bf16" else "alu", "kernel": kind_name,
+        "unit_of_work": "one step's launches of the kernel "
+                        f"({launches:g} per step: {', '.join(sorted(gemm_kinds))})",
+        "achieved": round(achieved, 1), "peak": burst, "unit": "TFLOP/s",
+        "frac": round(achieved / burst, 4),
+        "peak_note": f"bf16_tflops (burst) of {peaks_src} MEASURED_PEAKS.json",
+        "counted_flops_per_step": counted, "executed_flops_per_step": executed,
+        "executed_tflops": round(executed / (gemm_ms * 1e-3) / 1e12, 1),
+        "frac_executed_of_burst": round(executed / (gemm_ms * 1e-3) / 1e12 / burst, 4),
+        "frac_of_sustained": round(achieved / sust, 4),
+        "kernel_ms_per_step": round(gemm_ms, 4),
+        "share_of_step": round(gemm_ms / ms_per_step, 4),
+        "traffic": traffic, "algorithmic_bytes": algo,
+        "traffic_ratio": None if traffic is None else round(traffic / algo, 3),
+        "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch kind "
+                          f"(profiles/traffic_{w.name}.md) x launches per step"
+                          if traffic is not None else
+                          "none on file for the current kernel sources",
+    }
+
+
+def step_roofline(w, ms_per_step, peaks, peaks_src):
+    counted = w.flops_counted()
+    sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    t_burst = max(counted / (peaks["bf16_tflops"] * 1e12), algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9))
+    t_sust = max(counted / (sust * 1e12), algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9))
+    return {"counted_flops": counted,
+            "tflops": round(counted / (ms_per_step * 1e-3) / 1e12, 1),
+            "frac_of_burst": round(t_burst / (ms_per_step * 1e-3), 4),
+            "frac_of_sustained": round(t_sust / (ms_per_step * 1e-3), 4),
+            "cap_with_recompute": round((2 + int(w.compute_dW)) / (3 + int(w.compute_dW)), 4),
+            "peaks": peaks_src}
+
+
+def breakdown(per_kind, steps, ms_per_step):
+    total = sum(v[0] for v in per_kind.values())
+    out = {k: {"ms_per_step": round(v[0] / steps, 4),
+               "launches_per_step": round(v[1] / steps, 2),
+               "share_of_kernel_time": round(v[0] / total, 4),
+               "executed_tflops": round(v[2] / (v[0] * 1e-3) / 1e12, 1) if v[2] else None}
+           for k, v in sorted(per_kind.items())}
+    return out, total / steps
+
+
 def run_ours(args):
     import torch.distributed as dist
 
@@ -259,38 +468,13 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=dev)
     w = ALL_WORKLOADS[args.workload].with_(seed=ALL_WORKLOADS[args.workload].seed + rank)
-    inp = make_inputs(w, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    case = Case(pkg, w, dev, stream)
+    inp, out, ws = case.inp, case.out, case.ws
     X, W, b, Q, lab = inp["X"], inp["W"], inp["b"], inp["Q"], inp["shift_labels"]
     tgt = inp.get("target")
-    dt_code = pkg.DTYPES[X.dtype]
-    compute_db = inp["compute_db"]
-
-    def api_call(out=None, workspace=None, check_status=False):
-        """The public Python API call a user makes for this workload."""
-        if w.ce:
-            return pkg.cross_entropy_forward_backward(
-                X, W, b, tgt, inp["ignore_index"], inp["temperature"], inp["reduction"],
-                compute_dW=inp["compute_dW"], compute_db=compute_db,
-                accum_fp32=inp["accum_fp32"], out=out, workspace=workspace,
-                check_status=check_status)
-        return pkg.forward_backward(X, W, b, Q, lab, inp["ignore_index"], inp["temperature"],
-                                    inp["eps"], inp["reduction"], compute_dW=inp["compute_dW"],
-                                    compute_db=compute_db, accum_fp32=inp["accum_fp32"],
-                                    out=out, workspace=workspace, check_status=check_status)
-
-    r0 = api_call(check_status=True)
-    ws = r0["workspace"]
-    out = {k: r0[k] for k in ("loss", "dX", "dW", "db")}
-    stream = torch.cuda.current_stream(dev)
+    compute_db = case.compute_db
     p = lambda t: None if t is None else t.data_ptr()
-    call_args = (p(X), p(W), p(b), p(Q), p(lab), inp["ignore_index"], w.BT, w.H, w.V, dt_code,
-                 inp["temperature"], inp["eps"], pkg.REDUCTIONS[inp["reduction"]],
-                 inp["compute_dW"], compute_db, inp["accum_fp32"], p(out["loss"]), p(out["dX"]),
-                 p(out["dW"]), p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
-    ce_args = (p(X), p(W), p(b), p(tgt), inp["ignore_index"], w.BT, w.H, w.V, dt_code,
-               inp["temperature"], pkg.REDUCTIONS[inp["reduction"]], inp["compute_dW"],
-               compute_db, inp["accum_fp32"], p(out["loss"]), p(out["dX"]), p(out["dW"]),
-               p(out["db"]), p(ws), ws.numel(), stream.cuda_stream)
 
     n_total = torch.zeros((), dtype=torch.int64, device=dev)
     mask = tgt if w.ce else lab
@@ -298,8 +482,7 @@ def run_ours(args):
 
     def step():
         if not args.dp:
-            s = (pkg.flkl_ce_forward_backward(*ce_args) if w.ce
-                 else pkg.flkl_forward_backward(*call_args))
+            s = case.call()
         else:
             # the data-parallel step of lm_head_projection_b200.dp, raw entry points
             s = pkg.flkl_count_valid(p(mask), w.BT, inp["ignore_index"], p(n_total),
@@ -307,8 +490,8 @@ def run_ours(args):
             if s == 0:
                 if world > 1:
                     dist.all_reduce(n_total)
-                s = (pkg.flkl_ce_forward_backward_dp(*ce_args, p(n_total)) if w.ce
-                     else pkg.flkl_forward_backward_dp(*call_args, p(n_total)))
+                s = (pkg.flkl_ce_forward_backward_dp(*case.ce_args, p(n_total)) if w.ce
+                     else pkg.flkl_forward_backward_dp(*case.kl_args, p(n_total)))
             if s == 0 and world > 1:
                 for t in exchanged:
                     dist.all_reduce(t)
@@ -319,7 +502,7 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
+    for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
@@ -331,77 +514,46 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     barrier()
+    clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1), dev)
     status = pkg.flkl_device_status(ws.data_ptr(), stream.cuda_stream)
     if status != 0:
         raise pkg.FlklError(status, "device status after the timed region")
-
-    # ---------------- per-launch breakdown: K profiled steps
-    cap = 256
-    events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap)]
-    for e in events:  # torch creates the CUDA event on its first record
-        e.record(stream)
-    torch.cuda.synchronize()
-    per_kind = {}  # kind -> [ms, launches, gemm flops]
-    launches_per_step = 0
-    for _ in range(args.steps):
-        st, kinds, flops, n = pkg.flkl_forward_backward_profiled(*call_args, events, cap,
-                                                                 ce_target=p(tgt))
-        if st != 0:
-            raise pkg.FlklError(st, "flkl_forward_backward_profiled")
-        launches_per_step = n
-        torch.cuda.synchronize()
-        for i, k in enumerate(kinds):
-            d = per_kind.setdefault(pkg.LAUNCH_KINDS[k], [0.0, 0, 0.0])
-            d[0] += events[2 * i].elapsed_time(events[2 * i + 1])
-            d[1] += 1
-            d[2] += flops[i]
-    clocks.stop()
     clk = clocks.summary()
-
-    total_prof_ms = sum(v[0] for v in per_kind.values())
-    dominant = max(per_kind, key=lambda k: per_kind[k][0])
-    peaks, peaks_src = load_peaks()
-    peak_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    dom_ms, dom_n, dom_flops = per_kind[dominant]
-    if dom_flops > 0:
-        achieved = dom_flops / (dom_ms * 1e-3) / 1e12  # = flops per launch / avg launch time
-        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_sust,
-                    "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
-                    "traffic": dram_traffic(w.name, dominant),
-                    "kernel": f"tc_group_kernel ({dominant} launches)",
-                    "flops_per_launch": dom_flops / dom_n,
-                    "avg_launch_ms": round(dom_ms / dom_n, 4),
-                    "peak_note": f"bf16_tflops_sustained of {peaks_src}",
-                    "share": round(dom_ms / total_prof_ms, 3)}
-    else:
-        roofline = {"bound": "hbm", "achieved": None, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": None, "traffic": None, "kernel": dominant}
-    breakdown = {k: {"ms_per_step": round(v[0] / args.steps, 4), "launches_per_step":
-                     round(v[1] / args.steps, 2), "share": round(v[0] / total_prof_ms, 3),
-                     "tflops": round(v[2] / (v[0] * 1e-3) / 1e12, 1) if v[2] else None}
-                 for k, v in sorted(per_kind.items())}
-
     ms_per_step = ms / args.steps
-    tokens = w.BT * world
-    value = tokens / (ms_per_step * 1e-3)
-    counted = w.flops_counted()
-    step_tflops = counted / (ms_per_step * 1e-3) / 1e12
-    roof_time = max(counted / (peaks["bf16_tflops"] * 1e12),
-                    (algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9)))
-    step_roofline = {"counted_flops": counted, "tflops": round(step_tflops, 1),
-                     "frac_of_burst": round(roof_time / (ms_per_step * 1e-3), 4),
-                     "frac_of_sustained": round(
-                         max(counted / (peak_sust * 1e12),
-                             algorithmic_bytes(w) / (peaks["hbm_gbs"] * 1e9))
-                         / (ms_per_step * 1e-3), 4),
-                     "peaks": peaks_src}
+
+    # ---------------- per-launch breakdown: K more steps through the profiled
+    # entry, back to back as in the timed region (no synchronisation between
+    # steps), with the in-kernel SM clock sampled next to them
+    trace_n = 4096
+    trace_iv = max(1000, int(ms_per_step * args.steps * 1e6 * 1.5 / trace_n))
+    trace = torch.zeros(2 * trace_n, dtype=torch.int64, device=dev)
+    side = torch.cuda.Stream(dev)
+    torch.cuda.synchronize()
+    pkg.flkl_clock_trace(trace.data_ptr(), trace_n, trace_iv, side.cuda_stream)
+    per_kind, launches_per_step, prof_ms = case.profiled_steps(args.steps)
+    torch.cuda.synchronize()
+    sm_clock = sm_clock_summary(trace, prof_ms * args.steps)
+    if pkg.flkl_device_status(ws.data_ptr(), stream.cuda_stream) != 0:
+        raise pkg.FlklError(4, "device status after the profiled steps")
+    kinds, kernel_sum = breakdown(per_kind, args.steps, ms_per_step)
+    peaks, peaks_src = load_peaks()
+    roofline = kernel_roofline(w, per_kind, args.steps, peaks, peaks_src, ms_per_step)
+    sroof = step_roofline(w, ms_per_step, peaks, peaks_src)
+    breakdown_check = {
+        "profiled_ms_per_step": round(prof_ms, 4),
+        "kernel_sum_ms_per_step": round(kernel_sum, 4),
+        "kernel_sum_over_timed_step": round(kernel_sum / ms_per_step, 4),
+        "note": "the profiled steps run back to back like the timed ones; the kernel sum "
+                "leaves out the gaps between launches"}
 
     # ---------------- end to end: batch from pinned host memory, loss back
     # End to end through the public API: every step's batch (X and the
@@ -435,8 +587,20 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    tokens = w.BT * world
     e2e = {"value": round(tokens / (e2e_ms / args.steps * 1e-3), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4}
+    del pipe
+
+    # ---------------- the other bf16 workloads, same process (rank 0, N = 1)
+    others = None
+    if (rank == 0 and world == 1 and not args.dp and not args.no_other_workloads
+            and args.workload == HEADLINE):
+        others = {}
+        for name in OTHER_WORKLOADS:
+            others[name] = measure_other(pkg, ALL_WORKLOADS[name], dev, stream, args,
+                                         peaks, peaks_src, gpu_index)
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -449,9 +613,11 @@ def run_ours(args):
                          f"inputs pre-converted to fp64, {dt:.1f} s"}
 
     if rank == 0:
+        value = tokens / (ms_per_step * 1e-3)
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.name, "global_batch": w.BT * world, "BT_per_gpu": w.BT,
@@ -460,14 +626,55 @@ def run_ours(args):
                        "temperature": w.temperature,
                        "parallelism": f"dp{world}" + ("-allreduce" if args.dp else "-replicas"),
                        "l2": "inputs larger than L2 (W, Q), no flush"},
-            "e2e": e2e, "roofline": roofline, "step_roofline": step_roofline,
-            "kernels": breakdown,
+            "e2e": e2e, "roofline": roofline, "step_roofline": sroof,
+            "kernels": kinds, "breakdown_check": breakdown_check,
             "gpu_launches": int((launches_per_step + (1 if args.dp else 0)) * args.steps),
-            "clocks": clk, "cpu_baseline": cpu,
+            "clocks": clk, "sm_clock_in_kernel_mhz": sm_clock,
+            "other_workloads": others, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+OTHER_WORKLOADS = ("bf16_bt2048_h4096_v128256_frozen_ignore_t2_sum",
+                   "bf16_bt4096_h4096_v128256_bias_mean_peaked",
+                   "bf16_bt8192_h4096_v151936_frozen")
+
+
+def measure_other(pkg, w, dev, stream, args, peaks, peaks_src, gpu_index):
+    """One more bf16 workload in the same process: 3 warm-up calls, then
+    min(K, 10) timed calls (CUDA events, inputs larger than L2), the in-kernel
+    SM clock next to them and nvidia-smi clocks during them."""
+    case = Case(pkg, w, dev, stream)
+    steps = max(1, min(args.steps, 10))
+    for _ in range(3):
+        if case.call() != 0:
+            raise pkg.FlklError(1, w.name)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_index)
+    time.sleep(0.3)
+    trace_n = 2048
+    est = 2.0 * w.flops_counted() / 1e15 * 1e3  # ms per step at 0.5 PFLOP/s, generous
+    trace_iv = max(1000, int(est * steps * 1e6 * 1.5 / trace_n))
+    trace = torch.zeros(2 * trace_n, dtype=torch.int64, device=dev)
+    side = torch.cuda.Stream(dev)
+    torch.cuda.synchronize()
+    pkg.flkl_clock_trace(trace.data_ptr(), trace_n, trace_iv, side.cuda_stream)
+    clocks.mark_start()
+    ms = timed_steps(case, steps)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    clocks.stop()
+    if pkg.flkl_device_status(case.ws.data_ptr(), stream.cuda_stream) != 0:
+        raise pkg.FlklError(4, w.name)
+    msps = ms / steps
+    res = {"steps": steps, "warmup": 3, "ms_per_step": round(msps, 4),
+           "tokens_per_s": round(w.BT / (msps * 1e-3), 1),
+           "step_roofline": step_roofline(w, msps, peaks, peaks_src),
+           "clocks": clocks.summary(), "sm_clock_in_kernel_mhz": sm_clock_summary(trace, ms)}
+    del case
+    return res
 
 
 def algorithmic_bytes(w) -> float:
@@ -571,12 +778,14 @@ def run_norm(args):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     torch.cuda.synchronize()
+    clocks.mark_start()
     for a, b in evs:
         flush.zero_()
         a.record(stream)
         step()
         b.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     clocks.stop()
     if pkg.flkl_norm_device_status(stream0.cuda_stream) != 0:
         raise pkg.FlklError(4, "norm kernel wait")
@@ -662,11 +871,13 @@ def run_logprob(args):
     clocks = ClockSampler(0)
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     clocks.stop()
     if pkg.flkl_device_status(p(ws), stream.cuda_stream) != 0:
         raise pkg.FlklError(4, "device status after the timed region")
@@ -742,11 +953,13 @@ def run_jsd(args):
     clocks = ClockSampler(0)
     time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark_end()
     clocks.stop()
     if pkg.flkl_device_status(p(ws), stream.cuda_stream) != 0:
         raise pkg.FlklError(4, "device status after the timed region")
@@ -782,6 +995,61 @@ def run_jsd(args):
                          "sample": f"{rows} rows, fp64 numpy, {t_cpu:.1f} s"},
         "clocks": clocks.summary(),
     }
+    print(json.dumps(line), flush=True)
+
+
+def run_memory(args):
+    """Peak device memory of one fused forward + backward at the pages' head
+    shape (bf16, H=4096, V=128256, trained head) for BT = 1024, 2048, 4096:
+    through the C-ABI call (inputs, outputs and workspace) and through the
+    autograd module (loss.backward() filling X.grad and W.grad), with the head
+    gradient kept in bf16 and in fp32 (accum_dtype)."""
+    import lm_head_projection_b200 as pkg
+
+    dev = torch.device("cuda", 0)
+    mb = lambda n: round(n / 2**20, 1)
+    rows = []
+    for BT in (1024, 2048, 4096):
+        for accum in (False, True):
+            w = WORKLOADS[HEADLINE].with_(BT=BT, accum_fp32=accum)
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            base = torch.cuda.memory_allocated(dev)
+            inp = make_inputs(w, device=dev)
+            torch.cuda.synchronize()
+            in_bytes = torch.cuda.memory_allocated(dev) - base
+            torch.cuda.reset_peak_memory_stats(dev)
+            r = pkg.forward_backward(inp["X"], inp["W"], None, inp["Q"], compute_dW=True,
+                                     accum_fp32=accum, check_status=True)
+            torch.cuda.synchronize()
+            call_peak = torch.cuda.max_memory_allocated(dev) - base
+            ws = r["workspace"].numel()
+            out_bytes = sum(t.numel() * t.element_size() for k, t in r.items()
+                            if k != "workspace" and t is not None)
+            del r
+            torch.cuda.synchronize()
+            torch.cuda.empty_cache()
+            torch.cuda.reset_peak_memory_stats(dev)
+            X = inp["X"].clone().requires_grad_()
+            Wp = inp["W"].clone().requires_grad_()
+            del inp["X"], inp["W"]
+            mod = pkg.FusedLinearKLDivLoss(accum_dtype=torch.float32 if accum else None)
+            loss = mod(Wp, X, inp["Q"])
+            loss.backward()
+            torch.cuda.synchronize()
+            module_peak = torch.cuda.max_memory_allocated(dev) - base
+            rows.append({"BT": BT, "head_grad": "fp32" if accum else "bf16",
+                         "inputs_mb": mb(in_bytes), "outputs_mb": mb(out_bytes),
+                         "workspace_mb": mb(ws), "call_peak_mb": mb(call_peak),
+                         "module_fwd_bwd_peak_mb": mb(module_peak)})
+            del X, Wp, loss, inp, mod
+    line = {"metric": "peak device memory of one fused fwd+bwd (MiB)", "unit": "MiB",
+            "higher_is_better": False, "n_gpus": 1, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "bf16_h4096_v128256_trained", "BT": [1024, 2048, 4096]},
+            "rows": rows,
+            "context": "the pages' fused kernel on an RTX 4060 Laptop: 4244 (BT 1024, "
+                       "benchmark harness), 4310 (BT 2048), 6594 (BT 4096) MB, another machine "
+                       "and implementation"}
     print(json.dumps(line), flush=True)
 
 
@@ -827,6 +1095,8 @@ if __name__ == "__main__":
     a = parse()
     if a.calls > 0:
         run_calls(a)
+    elif a.op == "memory":
+        run_memory(a)
     elif a.op == "jsd":
         run_jsd(a)
     elif a.op == "logprob":

@@ -233,6 +233,34 @@ FLKL_API flkl_status flkl_ce_forward_backward_dp(
     int compute_dW, int compute_db, int accum_fp32, float* loss, void* dX, void* dW, void* db,
     void* workspace, size_t workspace_bytes, void* stream, const int64_t* n_valid_total);
 
+/* Overlap of the data-parallel dW exchange with the remaining chunks.
+ *
+ * flkl_vocab_chunks: the vocabulary chunks of a call with these sizes and
+ * flags; returns their number n (0 for invalid sizes or BT = 0) and, when
+ * `bounds` is non-NULL, writes bounds[0..min(n, capacity)] (host int64):
+ * chunk c covers dW / db rows [bounds[c], bounds[c+1]).
+ *
+ * The _dp_events entries are flkl_forward_backward_dp /
+ * flkl_ce_forward_backward_dp that also record chunk_done[c] (a
+ * cudaEvent_t created by the caller) on `stream` as soon as the dW rows of
+ * chunk c are final, for c < n_events; a caller can then all-reduce those
+ * rows on another stream (after cudaStreamWaitEvent) while the later chunks
+ * run.  db and the loss are final only when the whole call is. */
+FLKL_API int flkl_vocab_chunks(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW,
+                               int compute_db, int64_t* bounds, int capacity);
+FLKL_API flkl_status flkl_forward_backward_dp_events(
+    const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
+    int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
+    float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
+    void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
+    const int64_t* n_valid_total, void** chunk_done, int n_events);
+FLKL_API flkl_status flkl_ce_forward_backward_dp_events(
+    const void* X, const void* W, const void* b, const int64_t* target, int64_t ignore_index,
+    int64_t BT, int64_t H, int64_t V, int dtype, float temperature, int reduction,
+    int compute_dW, int compute_db, int accum_fp32, float* loss, void* dX, void* dW, void* db,
+    void* workspace, size_t workspace_bytes, void* stream, const int64_t* n_valid_total,
+    void** chunk_done, int n_events);
+
 /* Gradient-in-forward scaling for autograd (the FusedLinearKLDivLoss page,
  * Details, bullet 3: the gradients come from the forward call; the backward
  * only applies the incoming gradient of the loss):
@@ -382,6 +410,16 @@ FLKL_API void flkl_set_wait_limit_ms(unsigned int ms);
  * writes the resulting status code (FLKL_ERR_TIMEOUT expected) to the device
  * int *status_out.  Touches no other memory. */
 FLKL_API flkl_status flkl_wait_selftest(int* status_out, unsigned int limit_ms, void* stream);
+
+/* Measurement helper (not part of the loss): one thread samples the SM
+ * clock counter and the global nanosecond timer every interval_ns,
+ * n_samples times, writing (globaltimer, clock64) pairs to out[2i],
+ * out[2i+1] (device uint64 [2 * n_samples]).  Launched on `stream`, usually
+ * a side stream next to the kernels whose SM clock is wanted; it holds one
+ * thread of one SM for n_samples * interval_ns and ends by itself.
+ * n_samples in [1, 2^24], interval_ns in [1000, 10^8]. */
+FLKL_API flkl_status flkl_clock_trace(uint64_t* out, int n_samples, unsigned int interval_ns,
+                                      void* stream);
 
 /* Static text for a status code. */
 FLKL_API const char* flkl_status_string(int status);

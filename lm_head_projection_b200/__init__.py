@@ -26,7 +26,8 @@ __all__ = [
     "flkl_ce_forward_backward_dp", "count_valid", "flkl_selective_logprob_forward",
     "flkl_selective_logprob_backward", "selective_logprob", "SelectiveLogProb",
     "flkl_jsd_workspace_size", "flkl_jsd_forward_backward", "jsd_forward_backward",
-    "FusedLinearJSDLoss", "flkl_scale_cast",
+    "FusedLinearJSDLoss", "flkl_scale_cast", "flkl_clock_trace", "flkl_vocab_chunks",
+    "flkl_forward_backward_dp_events", "flkl_ce_forward_backward_dp_events",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -111,6 +112,17 @@ def _lib():
         lib.flkl_scale_cast.restype = c.c_int
         lib.flkl_scale_cast.argtypes = [c.c_void_p, c.c_int, c.c_void_p, c.c_int, c.c_int64,
                                         c.c_void_p, c.c_void_p]
+        lib.flkl_clock_trace.restype = c.c_int
+        lib.flkl_clock_trace.argtypes = [c.c_void_p, c.c_int, c.c_uint, c.c_void_p]
+        lib.flkl_vocab_chunks.restype = c.c_int
+        lib.flkl_vocab_chunks.argtypes = [c.c_int64, c.c_int64, c.c_int64, c.c_int, c.c_int,
+                                          c.c_int, c.c_void_p, c.c_int]
+        lib.flkl_forward_backward_dp_events.restype = c.c_int
+        lib.flkl_forward_backward_dp_events.argtypes = list(
+            lib.flkl_forward_backward.argtypes) + [c.c_void_p, c.c_void_p, c.c_int]
+        lib.flkl_ce_forward_backward_dp_events.restype = c.c_int
+        lib.flkl_ce_forward_backward_dp_events.argtypes = list(
+            lib.flkl_ce_forward_backward.argtypes) + [c.c_void_p, c.c_void_p, c.c_int]
         lib.flkl_count_valid.restype = c.c_int
         lib.flkl_count_valid.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_void_p]
         lib.flkl_forward_backward_noalloc.restype = c.c_int
@@ -314,6 +326,47 @@ def flkl_scale_cast(src, src_dtype, dst, dst_dtype, n, scale, stream=None) -> in
                                   stream)
 
 
+def flkl_clock_trace(out_ptr, n_samples, interval_ns, stream=None) -> int:
+    return _lib().flkl_clock_trace(out_ptr, int(n_samples), int(interval_ns), stream)
+
+
+def flkl_vocab_chunks(BT, H, V, dtype, compute_dW, compute_db) -> list:
+    """Row bounds of the vocabulary chunks of a call: [b0=0, b1, ..., bn=V]
+    (chunk c covers dW rows [b_c, b_{c+1})); [] for BT = 0."""
+    n = _lib().flkl_vocab_chunks(int(BT), int(H), int(V), int(dtype), int(bool(compute_dW)),
+                                 int(bool(compute_db)), None, 0)
+    if n <= 0:
+        return []
+    b = (ctypes.c_int64 * (n + 1))()
+    _lib().flkl_vocab_chunks(int(BT), int(H), int(V), int(dtype), int(bool(compute_dW)),
+                             int(bool(compute_db)), b, n)
+    return [int(b[i]) for i in range(n + 1)]
+
+
+def _event_array(events):
+    """cudaEvent_t handles of torch.cuda.Event objects; torch creates the CUDA
+    event on its first record, so an event never recorded is recorded once
+    here (on the current stream) first."""
+    for e in events:
+        if not e.cuda_event:
+            e.record()
+    return (ctypes.c_void_p * max(1, len(events)))(*[e.cuda_event for e in events])
+
+
+def flkl_forward_backward_dp_events(*args_and_events):
+    """flkl_forward_backward_dp's arguments, then n_valid_total, then a list of
+    recorded-once torch.cuda.Event (chunk_done[c])."""
+    *args, n_total, events = args_and_events
+    return _lib().flkl_forward_backward_dp_events(*args, n_total, _event_array(events),
+                                                  len(events))
+
+
+def flkl_ce_forward_backward_dp_events(*args_and_events):
+    *args, n_total, events = args_and_events
+    return _lib().flkl_ce_forward_backward_dp_events(*args, n_total, _event_array(events),
+                                                     len(events))
+
+
 def flkl_device_status(workspace_ptr, stream=None) -> int:
     return _lib().flkl_device_status(workspace_ptr, stream)
 
@@ -401,14 +454,18 @@ def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
                      compute_dW: bool = True, compute_db: bool = False, accum_fp32: bool = True,
                      out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
                      stream: Optional[torch.cuda.Stream] = None, check_status: bool = False,
-                     n_valid_total: Optional[torch.Tensor] = None) -> dict:
+                     n_valid_total: Optional[torch.Tensor] = None,
+                     chunk_events: Optional[list] = None) -> dict:
     """Loss and gradients in one call on the current CUDA stream.
 
     Allocates outputs (and the workspace) with torch unless given in ``out`` /
     ``workspace``; returns ``{"loss", "dX", "dW", "db"}`` (None for the ones
     not asked for).  Raises FlklError on a non-OK status.  ``n_valid_total``
     (a device int64 scalar) replaces the batch's kept-row count in the
-    divisor: the data-parallel form (see :mod:`.dp`).
+    divisor: the data-parallel form (see :mod:`.dp`); with it,
+    ``chunk_events`` (torch.cuda.Event, one per vocabulary chunk, see
+    :func:`flkl_vocab_chunks`) are recorded as each chunk's dW rows become
+    final.
     """
     if reduction not in REDUCTIONS:
         raise ValueError(f"unknown reduction {reduction!r}")
@@ -439,7 +496,10 @@ def forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional[torch.Tensor]
             workspace.numel(), st.cuda_stream)
     if n_valid_total is not None:
         _check_dev("n_valid_total", n_valid_total, torch.int64, (), dev)
-        status = flkl_forward_backward_dp(*args, _ptr(n_valid_total))
+        if chunk_events is not None:
+            status = flkl_forward_backward_dp_events(*args, _ptr(n_valid_total), chunk_events)
+        else:
+            status = flkl_forward_backward_dp(*args, _ptr(n_valid_total))
     else:
         status = flkl_forward_backward(*args)
     if status != FLKL_OK:
@@ -517,7 +577,8 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
                                    workspace: Optional[torch.Tensor] = None,
                                    stream: Optional[torch.cuda.Stream] = None,
                                    check_status: bool = False,
-                                   n_valid_total: Optional[torch.Tensor] = None) -> dict:
+                                   n_valid_total: Optional[torch.Tensor] = None,
+                                   chunk_events: Optional[list] = None) -> dict:
     """Fused linear + cross-entropy (one-hot teacher at ``target``) in one call.
     ``reduction="batchmean"`` divides by the kept rows (torch's cross_entropy
     "mean").  Same outputs and conventions as :func:`forward_backward`."""
@@ -547,7 +608,11 @@ def cross_entropy_forward_backward(X: torch.Tensor, W: torch.Tensor, b: Optional
             _ptr(dX), _ptr(dW), _ptr(db), _ptr(workspace), workspace.numel(), st.cuda_stream)
     if n_valid_total is not None:
         _check_dev("n_valid_total", n_valid_total, torch.int64, (), dev)
-        status = flkl_ce_forward_backward_dp(*args, _ptr(n_valid_total))
+        if chunk_events is not None:
+            status = flkl_ce_forward_backward_dp_events(*args, _ptr(n_valid_total),
+                                                        chunk_events)
+        else:
+            status = flkl_ce_forward_backward_dp(*args, _ptr(n_valid_total))
     else:
         status = flkl_ce_forward_backward(*args)
     if status != FLKL_OK:

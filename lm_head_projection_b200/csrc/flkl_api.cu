@@ -273,6 +273,13 @@ struct Phases {
   bool backward = true;
   float* logp = nullptr;         // forward: per-row output instead of the loss
   const float* dlogp = nullptr;  // backward: per-row upstream gradients
+  // data-parallel overlap: event c is recorded on the call's stream once the
+  // dW rows of vocabulary chunk c are final (c < n_chunk_events)
+  cudaEvent_t* chunk_done = nullptr;
+  int n_chunk_events = 0;
+  void chunk_finished(long long c, cudaStream_t st) const {
+    if (chunk_done != nullptr && c < n_chunk_events) cudaEventRecord(chunk_done[c], st);
+  }
 };
 
 // Merge of the statistics into row values, then the reduced loss and / or the
@@ -398,8 +405,11 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     L.mix = 0;  // problems in sequence (interleaving pass-2 and dW tiles measured slower)
     double f = 2.0 * BT * static_cast<double>(Vw) * H * (1 + (compute_dW ? 1 : 0));
     if (c + 1 < P.nchunks) f += 2.0 * BT * static_cast<double>(chunk_w(c + 1)) * H;
-    Rec r_(rec, 9, f);
-    FLKL_CUDA(launch_group(maps, L, st));
+    {
+      Rec r_(rec, 9, f);
+      FLKL_CUDA(launch_group(maps, L, st));
+    }
+    ph.chunk_finished(c, st);
   }
   if (compute_db) {
     Rec r_(rec, 7);
@@ -460,6 +470,7 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
                         256, 0, st>>>(G, 1, ldg, X, 1, H, Vw, H, BT, nullptr, dW, H, c0, 4);
       FLKL_CUDA(cudaGetLastError());
     }
+    ph.chunk_finished(c, st);
     const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
     // dX[r][h] (+)= sum_v G[r][v] W[c0 + v][h]
     Rec r_(rec, 6, 2.0 * BT * static_cast<double>(Vw) * H);
@@ -1082,6 +1093,16 @@ flkl_status flkl_scale_cast(const void* src, int src_dtype, void* dst, int dst_d
   return cudaGetLastError() == cudaSuccess ? FLKL_OK : FLKL_ERR_CUDA;
 }
 
+flkl_status flkl_clock_trace(uint64_t* out, int n_samples, unsigned int interval_ns,
+                             void* stream) {
+  if (out == nullptr || n_samples < 1 || n_samples > (1 << 24) || interval_ns < 1000u ||
+      interval_ns > 100000000u)
+    return FLKL_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(out) & 7u) return FLKL_ERR_UNSUPPORTED;
+  k_clock_trace<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(out, n_samples, interval_ns);
+  return cudaGetLastError() == cudaSuccess ? FLKL_OK : FLKL_ERR_CUDA;
+}
+
 flkl_status flkl_count_valid(const int64_t* labels, int64_t BT, int64_t ignore_index,
                              int64_t* count, void* stream) {
   if (count == nullptr || BT < 0) return FLKL_ERR_INVALID_ARG;
@@ -1123,6 +1144,55 @@ flkl_status flkl_ce_forward_backward_dp(const void* X, const void* W, const void
                                temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
                                BT > 0 ? target : nullptr, n_valid_total);
+}
+
+int flkl_vocab_chunks(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW,
+                      int compute_db, int64_t* bounds, int capacity) {
+  Plan p;
+  if (!make_plan(BT, H, V, dtype, compute_dW, compute_db, p)) return 0;
+  if (BT == 0) return 0;  // no launch, no chunk
+  if (bounds != nullptr) {
+    for (long long c = 0; c <= p.nchunks && c <= capacity; ++c)
+      bounds[c] = std::min<long long>(c * p.Vc, V);
+  }
+  return static_cast<int>(p.nchunks);
+}
+
+flkl_status flkl_forward_backward_dp_events(
+    const void* X, const void* W, const void* b, const void* Q, const int64_t* shift_labels,
+    int64_t ignore_index, int64_t BT, int64_t H, int64_t V, int dtype, float temperature,
+    float eps, int reduction, int compute_dW, int compute_db, int accum_fp32, float* loss,
+    void* dX, void* dW, void* db, void* workspace, size_t workspace_bytes, void* stream,
+    const int64_t* n_valid_total, void** chunk_done, int n_events) {
+  if (n_valid_total == nullptr || (reinterpret_cast<uintptr_t>(n_valid_total) & 7u))
+    return FLKL_ERR_INVALID_ARG;
+  if (n_events < 0 || (n_events > 0 && chunk_done == nullptr)) return FLKL_ERR_INVALID_ARG;
+  Phases ph;
+  ph.chunk_done = reinterpret_cast<cudaEvent_t*>(chunk_done);
+  ph.n_chunk_events = n_events;
+  return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
+                               temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
+                               nullptr, n_valid_total, ph);
+}
+
+flkl_status flkl_ce_forward_backward_dp_events(
+    const void* X, const void* W, const void* b, const int64_t* target, int64_t ignore_index,
+    int64_t BT, int64_t H, int64_t V, int dtype, float temperature, int reduction,
+    int compute_dW, int compute_db, int accum_fp32, float* loss, void* dX, void* dW, void* db,
+    void* workspace, size_t workspace_bytes, void* stream, const int64_t* n_valid_total,
+    void** chunk_done, int n_events) {
+  if (BT > 0 && target == nullptr) return FLKL_ERR_INVALID_ARG;
+  if (n_valid_total == nullptr || (reinterpret_cast<uintptr_t>(n_valid_total) & 7u))
+    return FLKL_ERR_INVALID_ARG;
+  if (n_events < 0 || (n_events > 0 && chunk_done == nullptr)) return FLKL_ERR_INVALID_ARG;
+  Phases ph;
+  ph.chunk_done = reinterpret_cast<cudaEvent_t*>(chunk_done);
+  ph.n_chunk_events = n_events;
+  return forward_backward_impl(X, W, b, nullptr, nullptr, ignore_index, BT, H, V, dtype,
+                               temperature, 0.f, reduction, compute_dW, compute_db, accum_fp32,
+                               loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
+                               BT > 0 ? target : nullptr, n_valid_total, ph);
 }
 
 size_t flkl_jsd_workspace_size(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype,

@@ -253,4 +253,18 @@ __global__ void __launch_bounds__(256) k_scale_cast(const TS* src, TD* dst, long
   }
 }
 
+// One thread: (globaltimer, clock64) every interval_ns, n samples.  Each wait
+// ends when the global timer passes its target, so the kernel runs for about
+// n * interval_ns.
+__global__ void k_clock_trace(uint64_t* out, int n, unsigned int interval_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (int i = 0; i < n; ++i) {
+    const uint64_t target = t0 + static_cast<uint64_t>(i) * interval_ns;
+    uint64_t t = globaltimer_ns();
+    while (t < target) t = globaltimer_ns();
+    out[2 * i] = t;
+    out[2 * i + 1] = static_cast<uint64_t>(clock64());
+  }
+}
+
 }  // namespace flkl

@@ -11,6 +11,11 @@ gradients, so one step is:
 3. all-reduce the loss, dW and db (sum).  dX needs no exchange: each rank's
    dX rows are the whole batch's dX rows for its shard.
 
+With NCCL and a trained head, step 3 overlaps the call: the library records
+an event as each vocabulary chunk's dW rows become final, and those rows are
+all-reduced on a side stream while the later chunks run; the loss and db
+follow once the call ends, and the caller's stream waits for the exchange.
+
 The library itself runs no collective; the exchange is torch.distributed's.
 Every rank takes the same collective steps in the same order.
 """
@@ -22,7 +27,8 @@ from typing import Optional
 import torch
 import torch.distributed as dist
 
-from . import count_valid, cross_entropy_forward_backward, forward_backward
+from . import (DTYPES, count_valid, cross_entropy_forward_backward, flkl_vocab_chunks,
+               forward_backward)
 
 __all__ = ["DataParallelFusedLinearLoss"]
 
@@ -66,10 +72,13 @@ class DataParallelFusedLinearLoss:
             self._out_key = key
         return self.out
 
-    def _local(self, X, W, b, teacher, labels, n_total, compute_dW, compute_db) -> dict:
+    def _local(self, X, W, b, teacher, labels, n_total, compute_dW, compute_db,
+               chunk_events=None) -> dict:
         out = self._reusable_out(X, W, b, compute_dW, compute_db)
         common = dict(compute_dW=compute_dW, compute_db=compute_db, accum_fp32=self.accum_fp32,
                       out=out, workspace=self.workspace, n_valid_total=n_total)
+        if chunk_events is not None:
+            common["chunk_events"] = chunk_events
         if self.kind == "ce":
             r = cross_entropy_forward_backward(X, W, b, teacher, self.ignore_index,
                                                self.temperature, self.reduction, **common)
@@ -94,7 +103,40 @@ class DataParallelFusedLinearLoss:
         mask = teacher if self.kind == "ce" else shift_labels
         n_total = self._count(mask, X.shape[0], X.device)
         self._all_reduce([n_total])
-        r = self._local(X, W, b, teacher, shift_labels, n_total, compute_dW, compute_db)
-        self._all_reduce([r[k] for k in ("loss", "dW", "db") if r[k] is not None])
+        bounds = self._overlap_bounds(X, W, compute_dW, compute_db)
+        if not bounds:
+            r = self._local(X, W, b, teacher, shift_labels, n_total, compute_dW, compute_db)
+            self._all_reduce([r[k] for k in ("loss", "dW", "db") if r[k] is not None])
+        else:
+            r = self._overlapped(X, W, b, teacher, shift_labels, n_total, compute_dW,
+                                 compute_db, bounds)
         return {"loss": r["loss"], "dX": r["dX"], "dW": r["dW"], "db": r["db"],
                 "n_valid_total": n_total}
+
+    # -- overlap of the dW exchange with the call (NCCL, trained head)
+    def _overlap_bounds(self, X, W, compute_dW, compute_db) -> list:
+        if not (compute_dW and X.is_cuda and dist.is_initialized()
+                and dist.get_backend(self.group) == "nccl"):
+            return []
+        return flkl_vocab_chunks(X.shape[0], X.shape[1], W.shape[0], DTYPES[X.dtype],
+                                 compute_dW, compute_db)
+
+    def _overlapped(self, X, W, b, teacher, labels, n_total, compute_dW, compute_db,
+                    bounds) -> dict:
+        main = torch.cuda.current_stream(X.device)
+        side = getattr(self, "_side", None)
+        if side is None or side.device != X.device:
+            side = self._side = torch.cuda.Stream(X.device)
+        events = [torch.cuda.Event() for _ in range(len(bounds) - 1)]
+        r = self._local(X, W, b, teacher, labels, n_total, compute_dW, compute_db,
+                        chunk_events=events)
+        done = torch.cuda.Event()
+        done.record(main)
+        with torch.cuda.stream(side):
+            for c, ev in enumerate(events):
+                side.wait_event(ev)
+                self._all_reduce([r["dW"][bounds[c]:bounds[c + 1]]])
+            side.wait_event(done)
+            self._all_reduce([r[k] for k in ("loss", "db") if r[k] is not None])
+        main.wait_stream(side)
+        return r

@@ -43,35 +43,86 @@ def test_dram_traffic_lookup_follows_the_kernel_sources():
     assert bench.dram_traffic("no_such_workload", "chunk") is None
 
 
-def _sampler_with(tmp_path, lines):
+def _sampler_with(tmp_path, lines, t0=None, t1=None):
     s = object.__new__(bench.ClockSampler)
     s.path = str(tmp_path / "clocks.csv")
     with open(s.path, "w") as f:
         f.write("\n".join(lines) + "\n")
     s.proc = object()  # a sampler that ran
+    s.t0, s.t1 = t0, t1
     return s
 
 
-def test_clock_summary_median_under_load_and_reasons(tmp_path):
-    rows = ["0, 1965, 1965, 300.0, 0x0, Not Active, Not Active, Not Active, Not Active"] * 4
-    rows += ["0, 1400, 1965, 999.0, 0x4, Not Active, Not Active, Not Active, Active"] * 8
-    s = _sampler_with(tmp_path, rows)
-    r = s.summary()
+def _ts(sec):
+    import datetime
+    return datetime.datetime.fromtimestamp(sec).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+
+
+def test_clock_summary_keeps_the_timed_region_only(tmp_path):
+    t = 1_700_000_000.0
+    idle = [f"{_ts(t + 0.02 * i)}, 0, 1965, 1965, 300.0, 0x0, Not Active, Not Active, "
+            "Not Active, Not Active" for i in range(10)]
+    load = [f"{_ts(t + 0.2 + 0.02 * i)}, 0, 1400, 1965, 999.0, 0x4, Not Active, Not Active, "
+            "Not Active, Active" for i in range(8)]
+    after = [f"{_ts(t + 0.4 + 0.02 * i)}, 0, 1965, 1965, 300.0, 0x0, Not Active, Not Active, "
+             "Not Active, Not Active" for i in range(5)]
+    r = _sampler_with(tmp_path, idle + load + after, t0=t + 0.19, t1=t + 0.37).summary()
     assert r["sm_max_mhz"] == 1965.0
     assert r["reasons"] == ["sw_power_cap"]
-    assert r["samples"] == 12
-    assert 1400.0 <= r["sm_mhz"] <= 1965.0
+    assert r["samples"] == 8 and r["window"] == "timed region"
+    assert r["sm_mhz"] == 1400.0 and r["power_w_median"] == 999.0
 
 
-def test_clock_summary_reports_thermal_slowdown(tmp_path):
-    rows = ["0, 1200, 1965, 800.0, 0x40, Not Active, Active, Not Active, Not Active"] * 3
-    r = _sampler_with(tmp_path, rows).summary()
+def test_clock_summary_of_a_region_shorter_than_the_period(tmp_path):
+    t = 1_700_000_000.0
+    rows = [f"{_ts(t + 0.02 * i)}, 0, {1200 + i}, 1965, 800.0, 0x40, Not Active, Active, "
+            "Not Active, Not Active" for i in range(6)]
+    r = _sampler_with(tmp_path, rows, t0=t + 0.041, t1=t + 0.049).summary()
+    assert r["samples"] == 1 and r["sm_mhz"] == 1203.0
+    assert r["window"] == "first sample after the timed region"
     assert "hw_thermal_slowdown" in r["reasons"]
 
 
 def test_clock_summary_without_samples(tmp_path):
     r = _sampler_with(tmp_path, ["garbage"]).summary()
     assert r["sm_mhz"] is None and r["reasons"] == ["no samples"]
+
+
+def test_sm_clock_summary_from_a_trace():
+    import torch
+
+    # 1 ms apart, clock counter advancing 1500 cycles per microsecond
+    t = [1_000_000 * i for i in range(11)]
+    c = [1_500_000 * i for i in range(11)]
+    buf = torch.tensor([v for pair in zip(t, c) for v in pair], dtype=torch.int64)
+    r = bench.sm_clock_summary(buf, window_ms=5.5)
+    assert r["median"] == 1500 and r["samples"] == 5
+
+
+def test_kernel_roofline_counts_the_method_flops_against_the_burst_peak():
+    w = WORKLOADS["bf16_bt1024_h4096_v128256"]
+    g = 2.0 * w.BT * w.H * w.V
+    steps = 2
+    # per kind: [ms over all steps, launches, executed GEMM FLOPs]
+    per_kind = {"stats": [2 * 0.8, 2, 2 * g], "grad": [2 * 0.1, 2, 2 * g / 8],
+                "chunk": [2 * 2.4, 16, 2 * (g * 2 + g * 7 / 8)], "combine": [2 * 0.03, 2, 0.0]}
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    r = bench.kernel_roofline(w, per_kind, steps, peaks, "measured", 3.4)
+    assert r["kernel_ms_per_step"] == pytest.approx(3.3)
+    assert r["achieved"] == pytest.approx(round(3 * g / 3.3e-3 / 1e12, 1))
+    assert r["peak"] == 1600.0 and r["frac"] == pytest.approx(r["achieved"] / 1600.0, abs=1e-4)
+    assert r["executed_flops_per_step"] == pytest.approx(4 * g)
+    assert r["frac_executed_of_burst"] > r["frac"]
+    assert r["share_of_step"] == pytest.approx(3.3 / 3.4, abs=1e-4)
+
+
+def test_step_roofline_cap_and_fractions():
+    w = WORKLOADS["bf16_bt2048_h4096_v128256_frozen_ignore_t2_sum"]
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0}
+    ms = w.flops_counted() / 1600e12 * 1e3 * 2  # half of the burst roofline rate
+    r = bench.step_roofline(w, ms, peaks, "measured")
+    assert r["frac_of_burst"] == pytest.approx(0.5, abs=1e-4)
+    assert r["cap_with_recompute"] == pytest.approx(2 / 3, abs=1e-4)
 
 
 def test_max_over_ranks_without_a_group_is_the_value():

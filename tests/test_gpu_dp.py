@@ -151,3 +151,58 @@ def test_steps_of_changing_batch_size_get_buffers_of_their_own_size():
                     assert torch.equal(r[k], direct[k]), (BT, k)
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("kind", ["kl", "ce"])
+def test_chunk_events_and_overlapped_exchange_give_the_direct_call(kind):
+    """The vocabulary chunks reported by the library tile [0, V); the call
+    that records an event per chunk gives the plain call's bytes; and the
+    one-rank NCCL step whose dW exchange runs chunk by chunk on a side stream
+    (ordered by those events) gives the direct call's bytes."""
+    import torch.distributed as dist
+
+    import lm_head_projection_b200 as pkg
+    from lm_head_projection_b200.dp import DataParallelFusedLinearLoss
+
+    w = small_case(dtype="bf16", BT=300, H=256, V=4104, bias=True, ignore_frac=0.1,
+                   ce=(kind == "ce"), seed=6)
+    g = {k: (v.cuda() if isinstance(v, torch.Tensor) else v)
+         for k, v in make_inputs(w).items()}
+    bounds = pkg.flkl_vocab_chunks(w.BT, w.H, w.V, 1, True, True)
+    assert bounds[0] == 0 and bounds[-1] == w.V and len(bounds) >= 3
+    assert all(a < b for a, b in zip(bounds, bounds[1:]))
+    assert pkg.flkl_vocab_chunks(0, w.H, w.V, 1, True, True) == []
+    direct = _call(pkg, g)
+    n_total = pkg.count_valid(g["target"] if kind == "ce" else g["shift_labels"], w.BT)
+    events = [torch.cuda.Event() for _ in range(len(bounds) - 1)]
+    common = dict(compute_dW=True, compute_db=True, accum_fp32=True, n_valid_total=n_total,
+                  chunk_events=events, check_status=True)
+    if kind == "ce":
+        r = pkg.cross_entropy_forward_backward(g["X"], g["W"], g["b"], g["target"],
+                                               g["ignore_index"], g["temperature"],
+                                               g["reduction"], **common)
+    else:
+        r = pkg.forward_backward(g["X"], g["W"], g["b"], g["Q"], g["shift_labels"],
+                                 g["ignore_index"], g["temperature"], g["eps"], g["reduction"],
+                                 **common)
+    torch.cuda.synchronize()
+    for e in events:
+        assert e.query()  # every chunk's event was recorded and has completed
+    for k in ("loss", "dX", "dW", "db"):
+        assert torch.equal(r[k], direct[k]), k
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda:0"))
+    try:
+        loss = DataParallelFusedLinearLoss(kind, temperature=w.temperature, eps=w.eps)
+        assert loss._overlap_bounds(g["X"], g["W"], True, True) == bounds
+        teacher = g["target"] if kind == "ce" else g["Q"]
+        for _ in range(2):
+            out = loss.step(g["X"], g["W"], g["b"], teacher, g["shift_labels"],
+                            compute_dW=True, compute_db=True)
+            torch.cuda.synchronize()
+            for k in ("loss", "dX", "dW", "db"):
+                assert torch.equal(out[k], direct[k]), k
+    finally:
+        dist.destroy_process_group()
