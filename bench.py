@@ -317,17 +317,20 @@ class Case:
         return (pkg.flkl_ce_forward_backward(*self.ce_args) if self.w.ce
                 else pkg.flkl_forward_backward(*self.kl_args))
 
-    def profiled_steps(self, steps: int, cap: int = 32):
+    def profiled_steps(self, steps: int, cap: int = 32, before=None):
         """`steps` calls through the profiled entry, events around every
         launch, no synchronisation between calls (the same back-to-back launch
-        stream as the timed steps).  Returns per-kind [ms, launches, GEMM
-        FLOPs], the launches per call, and the elapsed ms per call from the
-        first event to the last."""
+        stream as the timed steps); `before()` runs right before the first
+        call (after the events are ready).  Returns per-kind [ms, launches,
+        GEMM FLOPs], the launches per call, and the elapsed ms per call from
+        the first event to the last."""
         pkg, st = self.pkg, self.stream
         events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * cap * steps)]
         for e in events:  # torch creates the CUDA event on its first record
             e.record(st)
         torch.cuda.synchronize()
+        if before is not None:
+            before()
         recs = []
         for i in range(steps):
             r = pkg.flkl_forward_backward_profiled(*self.kl_args,
@@ -370,12 +373,16 @@ def sm_clock_summary(buf: torch.Tensor, window_ms: float):
             "p90": round(mhz[(9 * len(mhz)) // 10]), "samples": len(mhz)}
 
 
-def timed_steps(case, steps, barrier=lambda: None):
+def timed_steps(case, steps, barrier=lambda: None, before=None):
     """Exactly `steps` calls between two events on the launch stream, with a
-    barrier and a synchronisation on both sides; returns elapsed ms."""
+    barrier and a synchronisation on both sides; `before()` runs after the
+    first synchronisation, right before the first event; returns elapsed
+    ms."""
     st = case.stream
     barrier()
     torch.cuda.synchronize()
+    if before is not None:
+        before()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(st)
     for _ in range(steps):
@@ -538,8 +545,9 @@ def run_ours(args):
     trace = torch.zeros(2 * trace_n, dtype=torch.int64, device=dev)
     side = torch.cuda.Stream(dev)
     torch.cuda.synchronize()
-    pkg.flkl_clock_trace(trace.data_ptr(), trace_n, trace_iv, side.cuda_stream)
-    per_kind, launches_per_step, prof_ms = case.profiled_steps(args.steps)
+    per_kind, launches_per_step, prof_ms = case.profiled_steps(
+        args.steps, before=lambda: pkg.flkl_clock_trace(trace.data_ptr(), trace_n, trace_iv,
+                                                        side.cuda_stream))
     torch.cuda.synchronize()
     sm_clock = sm_clock_summary(trace, prof_ms * args.steps)
     if pkg.flkl_device_status(ws.data_ptr(), stream.cuda_stream) != 0:
@@ -660,9 +668,9 @@ def measure_other(pkg, w, dev, stream, args, peaks, peaks_src, gpu_index):
     trace = torch.zeros(2 * trace_n, dtype=torch.int64, device=dev)
     side = torch.cuda.Stream(dev)
     torch.cuda.synchronize()
-    pkg.flkl_clock_trace(trace.data_ptr(), trace_n, trace_iv, side.cuda_stream)
     clocks.mark_start()
-    ms = timed_steps(case, steps)
+    ms = timed_steps(case, steps, before=lambda: pkg.flkl_clock_trace(
+        trace.data_ptr(), trace_n, trace_iv, side.cuda_stream))
     torch.cuda.synchronize()
     clocks.mark_end()
     clocks.stop()

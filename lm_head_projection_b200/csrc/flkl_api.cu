@@ -46,8 +46,9 @@ struct Plan {
   long long n_stat;            // column groups of the pass-1 statistics
   long long Vc, nchunks;
   long long db_groups;
-  long long n_counters;  // tile counters of the persistent launches
-  size_t off_cnt, off_st, off_rows, off_G, off_dx, off_db, total;
+  long long n_counters;  // tile counters of the persistent launches, then combine tickets
+  long long comb_rowblocks, comb_splits;  // grid of k_combine_split
+  size_t off_cnt, off_st, off_rows, off_cpart, off_G, off_dx, off_db, total;
   size_t g_stride;       // bytes between the two G staging buffers
 };
 
@@ -77,13 +78,20 @@ bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int 
   p.nchunks = cdiv(V, vc);
   p.db_groups = p.tc ? p.m_tiles * (TC_BM / 32) : p.m_tiles;
   size_t off = align256(sizeof(DevCtl));
-  p.n_counters = p.nchunks + 2;
+  // the merge of the statistics: about two blocks per SM of a 148-SM part,
+  // at least 16 column groups per split
+  p.comb_rowblocks = std::max<long long>(1, cdiv(BT, 32));
+  p.comb_splits = std::max<long long>(
+      1, std::min<long long>({cdiv(296, p.comb_rowblocks), 16, p.n_stat / 16}));
+  p.n_counters = p.nchunks + 2 + p.comb_rowblocks + 1;
   p.off_cnt = off;
   off += align256(size_t(p.n_counters) * 4);
   p.off_st = off;
   off += align256(size_t(5) * p.n_stat * BT * 4);
   p.off_rows = off;
   off += align256(size_t(4) * BT * 4);
+  p.off_cpart = off;
+  off += align256(size_t(5) * p.comb_splits * BT * 4);
   p.off_G = off;
   // two staging buffers on the tensor-core path: chunk c+1's gradient block
   // is produced while chunk c's is consumed
@@ -286,20 +294,24 @@ struct Phases {
 // per-row log-probabilities.
 cudaError_t finish_rows(const Plan& P, const float* stats, int BT, const int64_t* labels,
                         long long ignore_index, float T, DevCtl* ctl, float* lse2, float* coefS,
-                        float* coefQ, float* rowloss, float* loss, float* logp, cudaStream_t st,
-                        Recorder* rec) {
+                        float* coefQ, float* rowloss, float* loss, float* logp, uint8_t* ws,
+                        cudaStream_t st, Recorder* rec) {
   {
+    // merge, row values and (with `loss`) the reduced loss in one launch
     Rec r_(rec, 2);
-    k_combine<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kCombineWarps, 0, st>>>(
-        stats, static_cast<int>(P.n_stat), BT, labels, ignore_index, 1.f / T, ctl, lse2, coefS,
-        coefQ, rowloss);
+    int* tickets = reinterpret_cast<int*>(ws + P.off_cnt) + (P.nchunks + 2);
+    k_combine_split<<<dim3(static_cast<unsigned>(P.comb_rowblocks),
+                           static_cast<unsigned>(P.comb_splits)),
+                      32 * kCombSplitWarps, 0, st>>>(
+        stats, static_cast<int>(P.n_stat), BT, static_cast<int>(P.comb_splits), labels,
+        ignore_index, 1.f / T, ctl, reinterpret_cast<float*>(ws + P.off_cpart), tickets, lse2,
+        coefS, coefQ, rowloss, loss);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
+  if (logp == nullptr) return cudaSuccess;
   Rec r_(rec, 3);
-  if (loss != nullptr) k_loss<<<1, 1024, 0, st>>>(rowloss, BT, ctl, loss);
-  if (logp != nullptr)
-    k_neg_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(rowloss, BT, logp);
+  k_neg_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(rowloss, BT, logp);
   return cudaGetLastError();
 }
 
@@ -372,7 +384,7 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
       FLKL_CUDA(launch_group(maps, L, st));
     }
     FLKL_CUDA(finish_rows(P, stats, BT, labels, ignore_index, T, ctl, lse2, coefS, coefQ,
-                          rowloss, loss, ph.logp, st, rec));
+                          rowloss, loss, ph.logp, ws, st, rec));
   }
   if (!ph.backward) return FLKL_OK;
   FLKL_CUDA(upstream_coefs(ph.dlogp, target, BT, ignore_index, V, T, coefS, coefQ, st, rec));
@@ -447,7 +459,7 @@ flkl_status run_f32(const Plan& P, const float* X, const float* W, const float* 
       FLKL_CUDA(cudaGetLastError());
     }
     FLKL_CUDA(finish_rows(P, stats, BT, labels, ignore_index, T, ctl, lse2, coefS, coefQ,
-                          rowloss, loss, ph.logp, st, rec));
+                          rowloss, loss, ph.logp, ws, st, rec));
   }
   if (!ph.backward) return FLKL_OK;
   FLKL_CUDA(upstream_coefs(ph.dlogp, target, BT, ignore_index, V, T, coefS, coefQ, st, rec));
@@ -500,6 +512,8 @@ struct JsdPlan {
   bool tc;
   long long m_tiles, n_tiles, n_stat, Vc, nchunks, db_groups, n_counters;
   size_t off_cnt, off_st, off_rows, off_tgt, off_P, off_Q, off_G, off_dx, off_db, total;
+  size_t stage;     // bytes of one staging block (BT x Vc elements)
+  size_t off_part;  // tensor-core path: [2][n_stat][BT] fp32 partial sums of the loss sweep
 };
 
 constexpr int kJsdRows = 10;  // fp32 row arrays in the workspace
@@ -526,8 +540,9 @@ bool make_jsd_plan(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype, int 
   vc = std::min(vc, p.n_tiles * tile);
   p.Vc = vc;
   p.nchunks = cdiv(V, vc);
-  p.db_groups = cdiv(BT, kJsdRowGroup);
-  p.n_counters = 2 + 5 * p.nchunks;
+  // db partials per 32-row group: over whole 256-row tiles on the tensor-core path
+  p.db_groups = p.tc ? p.m_tiles * (TC_BM / 32) : cdiv(BT, kJsdRowGroup);
+  p.n_counters = 2 + 5 * p.nchunks + 2;
   size_t off = align256(sizeof(DevCtl));
   p.off_cnt = off;
   off += align256(size_t(p.n_counters) * 4);
@@ -537,13 +552,28 @@ bool make_jsd_plan(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype, int 
   off += align256(size_t(kJsdRows) * BT * 4);
   p.off_tgt = off;
   off += align256(size_t(BT) * 8);
-  // student and teacher probabilities of one chunk; the gradient block
-  // overwrites the student's in place
   const size_t stage = align256(size_t(BT) * vc * elem);
-  p.off_P = off;
-  p.off_Q = off + stage;
-  p.off_G = off;
-  off += 2 * stage;
+  p.stage = stage;
+  if (p.tc) {
+    // teacher probabilities of chunks c and c+1 (read by the student pass of
+    // chunk c while the teacher pass of chunk c+1 writes; the student pass of
+    // the gradient sweep overwrites chunk c's block with its gradient block),
+    // and the loss sweep's partial sums
+    p.off_Q = off;
+    p.off_P = off;
+    p.off_G = off;
+    off += 2 * stage;
+    p.off_part = off;
+    off += align256(size_t(2) * p.n_stat * BT * 4);
+  } else {
+    // student and teacher probabilities of one chunk; the gradient block
+    // overwrites the student's in place
+    p.off_P = off;
+    p.off_Q = off + stage;
+    p.off_G = off;
+    p.off_part = 0;
+    off += 2 * stage;
+  }
   p.off_dx = off;
   if (p.nchunks > 1) off += align256(size_t(BT) * H * 4);
   p.off_db = off;
@@ -579,14 +609,23 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
                        int BT, int H, int Ht, int V, float T, float beta, int compute_dW,
                        int compute_db, int accum_fp32, float* loss, __nv_bfloat16* dX, void* dW,
                        void* db, uint8_t* ws, cudaStream_t st) {
+  // Sequence (no probability block of the student ever reaches memory):
+  //   statistics passes of the teacher and of the student (log-sum-exps);
+  //   loss sweep: teacher probabilities of chunk c+1 into a staging block while
+  //     the student pass of chunk c forms p, m and the partial sums of
+  //     KL(P||M) and the row loss in its epilogue (reading the staged q);
+  //   K and the loss from the partial sums (fixed order);
+  //   gradient sweep: the same pairing, the student epilogue writing the
+  //     gradient block G of chunk c over the teacher block it reads, then
+  //     dX(c) and dW(c) from G.
   DevCtl* ctl = reinterpret_cast<DevCtl*>(ws);
   int* counters = reinterpret_cast<int*>(ws + P.off_cnt);
   float* stats = reinterpret_cast<float*>(ws + P.off_st);
   const JsdRows R = jsd_rows(reinterpret_cast<float*>(ws + P.off_rows), BT);
   int64_t* nt = reinterpret_cast<int64_t*>(ws + P.off_tgt);
-  __nv_bfloat16* Pb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_P);
-  __nv_bfloat16* Qb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_Q);
-  __nv_bfloat16* Gb = reinterpret_cast<__nv_bfloat16*>(ws + P.off_G);
+  __nv_bfloat16* Qs[2] = {reinterpret_cast<__nv_bfloat16*>(ws + P.off_Q),
+                          reinterpret_cast<__nv_bfloat16*>(ws + P.off_Q + P.stage)};
+  float* part = reinterpret_cast<float*>(ws + P.off_part);
   float* dxpart = reinterpret_cast<float*>(ws + P.off_dx);
   float* dbpart = compute_db ? reinterpret_cast<float*>(ws + P.off_db) : nullptr;
   const float t_scale = 1.4426950408889634f / T;
@@ -625,18 +664,72 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
         R.scrQ, R.scrL);
     return cudaGetLastError();
   };
-  // probabilities of one side over chunk c into `out` (the pass-2 epilogue
-  // with coefficients 1 and 0 and no teacher)
-  auto side_probs = [&](const Operand& mA, const Operand& mB, int Hk,
-                        const __nv_bfloat16* bias, const float* lse2, __nv_bfloat16* out,
-                        long long c) -> cudaError_t {
-    TcLaunch L = new_launch();
-    TcMaps maps{};
+  // teacher probabilities of chunk c into Qs[c & 1] (the pass-2 epilogue with
+  // coefficients 1 and 0 and no target)
+  auto add_teacher = [&](TcLaunch& L, TcMaps& maps, long long c) {
     const int c0 = chunk_c0(c);
-    L.grad = EpiGrad::Params{nullptr, bias, BT,     V,       c0,      ldg,     out,
-                             t_scale, lse2, R.ones, R.zeros, nullptr, nt};
-    add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), Hk, 1, mA, mB, 0, c0, 0);
-    return launch_group(maps, L, st);
+    L.grad = EpiGrad::Params{nullptr, bt,      BT,      V,       c0,      ldg,     Qs[c & 1],
+                             t_scale, R.lse2_t, R.ones, R.zeros, nullptr, nt};
+    add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), Ht, 1, mXt_k, mWt_k, 0, c0, 0);
+  };
+  // student pass of chunk c, reading Qs[c & 1]
+  auto add_student = [&](TcLaunch& L, TcMaps& maps, long long c, int grad) {
+    const int c0 = chunk_c0(c);
+    EpiJsd::Params& j = L.jsd;
+    j = EpiJsd::Params{};
+    j.bias = b;
+    j.BT = BT;
+    j.V = V;
+    j.c0 = c0;
+    j.ldg = ldg;
+    j.Qs = Qs[c & 1];
+    j.t_scale = t_scale;
+    j.lse2 = R.lse2_s;
+    j.beta = beta;
+    j.grad = grad;
+    j.part = part;
+    j.part_plane = static_cast<long long>(P.n_stat) * BT;
+    j.G = Qs[c & 1];  // the gradient block replaces the teacher block it is formed from
+    j.K = R.K;
+    j.rowscale = R.rowscale;
+    j.dbpart = grad ? dbpart : nullptr;
+    add_problem(L, maps, KIND_JSD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, c0, 0);
+  };
+  // the teacher pass of chunk 0 alone, then per chunk c: the student pass of
+  // chunk c (longer: with the teacher read) and the teacher pass of chunk c+1
+  auto sweep = [&](int grad) -> flkl_status {
+    {
+      TcLaunch L = new_launch();
+      TcMaps maps{};
+      add_teacher(L, maps, 0);
+      FLKL_CUDA(launch_group(maps, L, st));
+    }
+    for (long long c = 0; c < P.nchunks; ++c) {
+      {
+        TcLaunch L = new_launch();
+        TcMaps maps{};
+        add_student(L, maps, c, grad);
+        if (c + 1 < P.nchunks) add_teacher(L, maps, c + 1);
+        FLKL_CUDA(launch_group(maps, L, st));
+      }
+      if (!grad) continue;
+      const int c0 = chunk_c0(c), Vw = chunk_w(c);
+      Operand mG_k, mG_mn;
+      if (!make_operand(&mG_k, Qs[c & 1], Vw, BT, ldg, false) ||
+          !make_operand(&mG_mn, Qs[c & 1], Vw, BT, ldg, true))
+        return FLKL_ERR_CUDA;
+      TcLaunch L = new_launch();
+      TcMaps maps{};
+      const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
+      L.dx = EpiAccumRows::Params{dxpart, dX, H, BT, H, mode};
+      add_problem(L, maps, KIND_DX, BT, H, Vw, 0, mG_k, mW_mn, 0, 0, c0);
+      if (compute_dW) {
+        L.dw = EpiStoreRows::Params{dW, H, Vw, H, c0, accum_fp32};
+        add_problem(L, maps, KIND_DW, Vw, H, BT, 1, mG_mn, mX_mn);
+      }
+      FLKL_CUDA(launch_group(maps, L, st));
+    }
+    return FLKL_OK;
   };
 
   FLKL_CUDA(side_lse(mXt_k, mWt_k, Ht, bt, R.lse2_t));
@@ -644,39 +737,14 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
   k_jsd_init_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
       labels, BT, ignore_index, ctl, R.rowscale, R.K, R.L);
   FLKL_CUDA(cudaGetLastError());
-  for (long long c = 0; c < P.nchunks; ++c) {
-    FLKL_CUDA(side_probs(mXt_k, mWt_k, Ht, bt, R.lse2_t, Qb, c));
-    FLKL_CUDA(side_probs(mX_k, mW_k, H, b, R.lse2_s, Pb, c));
-    k_jsd_rows<__nv_bfloat16><<<static_cast<unsigned>(cdiv(int64_t(BT) * 32, 256)), 256, 0, st>>>(
-        Pb, Qb, ldg, BT, chunk_w(c), beta, R.K, R.L);
-    FLKL_CUDA(cudaGetLastError());
-  }
-  k_jsd_row_loss<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(R.L, R.rowscale, BT,
-                                                                         R.scrL);
+  flkl_status s = sweep(0);
+  if (s != FLKL_OK) return s;
+  k_jsd_sum_parts<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
+      part, static_cast<int>(P.n_stat), BT, R.rowscale, R.K, R.scrL);
   k_loss<<<1, 1024, 0, st>>>(R.scrL, BT, ctl, loss);
   FLKL_CUDA(cudaGetLastError());
-  for (long long c = 0; c < P.nchunks; ++c) {
-    const int c0 = chunk_c0(c), Vw = chunk_w(c);
-    FLKL_CUDA(side_probs(mXt_k, mWt_k, Ht, bt, R.lse2_t, Qb, c));
-    FLKL_CUDA(side_probs(mX_k, mW_k, H, b, R.lse2_s, Pb, c));
-    k_jsd_grad<__nv_bfloat16>
-        <<<dim3(static_cast<unsigned>(cdiv(Vw, 256)), static_cast<unsigned>(P.db_groups)), 256,
-           0, st>>>(Pb, Qb, ldg, BT, Vw, c0, V, beta, R.K, R.rowscale, Gb, dbpart);
-    FLKL_CUDA(cudaGetLastError());
-    Operand mG_k, mG_mn;
-    if (!make_operand(&mG_k, Gb, Vw, BT, ldg, false) || !make_operand(&mG_mn, Gb, Vw, BT, ldg, true))
-      return FLKL_ERR_CUDA;
-    TcLaunch L = new_launch();
-    TcMaps maps{};
-    const int mode = P.nchunks == 1 ? 0 : (c == 0 ? 1 : (c == P.nchunks - 1 ? 3 : 2));
-    L.dx = EpiAccumRows::Params{dxpart, dX, H, BT, H, mode};
-    add_problem(L, maps, KIND_DX, BT, H, Vw, 0, mG_k, mW_mn, 0, 0, c0);
-    if (compute_dW) {
-      L.dw = EpiStoreRows::Params{dW, H, Vw, H, c0, accum_fp32};
-      add_problem(L, maps, KIND_DW, Vw, H, BT, 1, mG_mn, mX_mn);
-    }
-    FLKL_CUDA(launch_group(maps, L, st));
-  }
+  s = sweep(1);
+  if (s != FLKL_OK) return s;
   if (compute_db) {
     k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
         dbpart, static_cast<int>(P.db_groups), V, db, accum_fp32);

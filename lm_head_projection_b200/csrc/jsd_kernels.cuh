@@ -82,6 +82,24 @@ __global__ void __launch_bounds__(256) k_jsd_rows(const T* __restrict__ P, const
   }
 }
 
+// Tensor-core path: K[r] and the row loss from the loss sweep's partial sums
+// part[0][g][r] (of p ln(p/m)) and part[1][g][r] (of the row loss), summed
+// over the column groups g in order; dropped rows get 0.
+__global__ void k_jsd_sum_parts(const float* __restrict__ part, int n_groups, int BT,
+                                const float* __restrict__ rowscale, float* __restrict__ K,
+                                float* __restrict__ rowloss) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= BT) return;
+  const size_t plane = static_cast<size_t>(n_groups) * BT;
+  float k = 0.f, l = 0.f;
+  for (int g = 0; g < n_groups; ++g) {
+    k += part[static_cast<size_t>(g) * BT + r];
+    l += part[plane + static_cast<size_t>(g) * BT + r];
+  }
+  K[r] = k;
+  rowloss[r] = rowscale[r] != 0.f ? l : 0.f;
+}
+
 // Row losses of kept rows (dropped rows 0) for the fixed-order reduction.
 __global__ void k_jsd_row_loss(const float* __restrict__ L, const float* __restrict__ rowscale,
                                int BT, float* __restrict__ rowloss) {

@@ -164,6 +164,130 @@ __global__ void __launch_bounds__(32 * kCombineWarps)
   }
 }
 
+// Online merge of one (max, sum) pair of base-2 softmax statistics.
+__device__ __forceinline__ void merge_ms(float& m, float& s, float tm, float ts) {
+  if (tm == -INFINITY) return;  // nothing to merge (also keeps -inf - -inf out)
+  const float nm = fmaxf(m, tm);
+  s = s * exp2f(m - nm) + ts * exp2f(tm - nm);
+  m = nm;
+}
+
+// Row values from the merged statistics of one row.
+__device__ __forceinline__ void finish_row(int row, float m, float s, float A, float B2, float S,
+                                           const int64_t* __restrict__ labels,
+                                           long long ignore_index, float invT, float sc,
+                                           float* __restrict__ lse2_out,
+                                           float* __restrict__ coefS, float* __restrict__ coefQ,
+                                           float* __restrict__ rowloss) {
+  const float LN2 = 0.693147180559945309f;
+  const float lse2 = m + log2f(s);
+  const bool keep = labels == nullptr || labels[row] != ignore_index;
+  lse2_out[row] = lse2;
+  coefS[row] = keep ? S * sc : 0.f;
+  coefQ[row] = keep ? sc : 0.f;
+  rowloss[row] = keep ? (LN2 * B2 - A * invT + LN2 * lse2 * S) : 0.f;
+}
+
+// The merge of k_combine spread over more blocks, with the loss sum fused:
+// grid (ceil(BT/32) row blocks, `splits`); block (row block, split) merges
+// groups [split*G/splits, (split+1)*G/splits) of its 32 rows (warp w takes
+// every 8th group, then warp 0 merges the 8 warp partials in warp order) into
+// part[5][splits][BT].  The last block of a row block to finish (ticket
+// tickets[row block]) merges the splits' partials in split order and writes
+// the row values; when `loss` is given, the last row block to finish (ticket
+// tickets[row blocks]) sums the row losses in a fixed order (fp64) into
+// *loss = sum / D.  Every merge and sum has a fixed order, so the results do
+// not depend on which block finishes last.  The tickets are zero at launch.
+constexpr int kCombSplitWarps = 8;
+__global__ void __launch_bounds__(32 * kCombSplitWarps)
+    k_combine_split(const float* __restrict__ st, int n_groups, int BT, int splits,
+                    const int64_t* __restrict__ labels, long long ignore_index, float invT,
+                    const DevCtl* __restrict__ ctl, float* part, int* tickets,
+                    float* __restrict__ lse2_out, float* __restrict__ coefS,
+                    float* __restrict__ coefQ, float* rowloss, float* loss) {
+  __shared__ float sp[kCombSplitWarps][5][32];
+  __shared__ double red[32 * kCombSplitWarps];
+  __shared__ int is_last;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = blockIdx.x * 32 + lane;
+  const int split = blockIdx.y;
+  const size_t plane = static_cast<size_t>(n_groups) * BT;
+  const int g0 = static_cast<int>((static_cast<long long>(split) * n_groups) / splits);
+  const int g1 = static_cast<int>((static_cast<long long>(split + 1) * n_groups) / splits);
+  float m = -INFINITY, s = 0.f, A = 0.f, B2 = 0.f, S = 0.f;
+  if (row < BT) {
+#pragma unroll 4
+    for (int g = g0 + w; g < g1; g += kCombSplitWarps) {
+      const size_t o = static_cast<size_t>(g) * BT + row;
+      merge_ms(m, s, st[o], st[o + plane]);
+      A += st[o + 2 * plane];
+      B2 += st[o + 3 * plane];
+      S += st[o + 4 * plane];
+    }
+  }
+  sp[w][0][lane] = m;
+  sp[w][1][lane] = s;
+  sp[w][2][lane] = A;
+  sp[w][3][lane] = B2;
+  sp[w][4][lane] = S;
+  __syncthreads();
+  const size_t pplane = static_cast<size_t>(splits) * BT;
+  if (w == 0 && row < BT) {
+    m = sp[0][0][lane];
+    s = sp[0][1][lane];
+    A = sp[0][2][lane];
+    B2 = sp[0][3][lane];
+    S = sp[0][4][lane];
+    for (int k = 1; k < kCombSplitWarps; ++k) {
+      merge_ms(m, s, sp[k][0][lane], sp[k][1][lane]);
+      A += sp[k][2][lane];
+      B2 += sp[k][3][lane];
+      S += sp[k][4][lane];
+    }
+    const size_t o = static_cast<size_t>(split) * BT + row;
+    part[o] = m;
+    part[o + pplane] = s;
+    part[o + 2 * pplane] = A;
+    part[o + 3 * pplane] = B2;
+    part[o + 4 * pplane] = S;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&tickets[blockIdx.x], 1) == splits - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (w == 0 && row < BT) {
+    m = -INFINITY;
+    s = A = B2 = S = 0.f;
+    for (int k = 0; k < splits; ++k) {
+      const size_t o = static_cast<size_t>(k) * BT + row;
+      merge_ms(m, s, __ldcg(part + o), __ldcg(part + o + pplane));
+      A += __ldcg(part + o + 2 * pplane);
+      B2 += __ldcg(part + o + 3 * pplane);
+      S += __ldcg(part + o + 4 * pplane);
+    }
+    finish_row(row, m, s, A, B2, S, labels, ignore_index, invT, ctl->scale, lse2_out, coefS,
+               coefQ, rowloss);
+  }
+  if (loss == nullptr) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&tickets[gridDim.x], 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < BT; i += blockDim.x) acc += static_cast<double>(__ldcg(rowloss + i));
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if (static_cast<int>(threadIdx.x) < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *loss = static_cast<float>(red[0] * static_cast<double>(ctl->invD));
+}
+
 // loss = (sum of row losses) / D, summed in a fixed order (fp64 partials).
 __global__ void __launch_bounds__(1024) k_loss(const float* __restrict__ rowloss, int BT,
                                                const DevCtl* __restrict__ ctl, float* loss) {

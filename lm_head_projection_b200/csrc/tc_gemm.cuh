@@ -144,6 +144,16 @@ __device__ __forceinline__ void load_chunk32(const __nv_bfloat16* rowp, bool rv,
     u[j] = (rv && cc < limit) ? ld_nc_v4(rowp + cc) : make_uint4(0, 0, 0, 0);
   }
 }
+// load_chunk32 with coherent loads, for data the same kernel overwrites.
+__device__ __forceinline__ void load_chunk32_rw(const __nv_bfloat16* rowp, bool rv, int col0,
+                                                int limit, uint4 (&u)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int cc = col0 + 8 * j;
+    u[j] = (rv && cc < limit) ? *reinterpret_cast<const uint4*>(rowp + cc)
+                              : make_uint4(0, 0, 0, 0);
+  }
+}
 // Same 32 bias values for every lane of the warp (one broadcast request).
 __device__ __forceinline__ void load_bias32(const __nv_bfloat16* bias, int col0, int V,
                                             float (&bv)[32]) {
@@ -206,18 +216,35 @@ struct EpiStats {
 #pragma unroll
         for (int i = 0; i < 32; ++i) q[i] = (col0 + i == y) ? 1.f : 0.f;
       }
-      load_bias32(p.bias, col0, p.V, bv);
       tmem_ld32(taddr + c * 32, z);
-      float cm = -INFINITY;
+      if (p.bias != nullptr) {  // warp-uniform
+        load_bias32(p.bias, col0, p.V, bv);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool ok = (col0 + i) < p.V;
-        const float zz = z[i] + bv[i];
-        z[i] = ok ? zz * p.t_scale : -INFINITY;
-        cm = fmaxf(cm, z[i]);
-        A = fmaf(q[i], zz, A);
-        S += q[i];
-        B2 += (q[i] != 0.f) ? q[i] * __log2f(fmaxf(q[i], qmin)) : 0.f;
+        for (int i = 0; i < 32; ++i) z[i] += bv[i];
+      }
+      float cm = -INFINITY;
+      // q = 0 adds q * log2(qmin) = 0 (qmin >= FLT_MIN keeps the logarithm finite)
+      if (col0 + 32 <= p.V) {  // warp-uniform: every column of the chunk is a vocabulary entry
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float zz = z[i];
+          z[i] = zz * p.t_scale;
+          cm = fmaxf(cm, z[i]);
+          A = fmaf(q[i], zz, A);
+          S += q[i];
+          B2 += q[i] * __log2f(fmaxf(q[i], qmin));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool ok = (col0 + i) < p.V;
+          const float zz = z[i];
+          z[i] = ok ? zz * p.t_scale : -INFINITY;
+          cm = fmaxf(cm, z[i]);
+          A = fmaf(q[i], zz, A);
+          S += q[i];
+          B2 += q[i] * __log2f(fmaxf(q[i], qmin));
+        }
       }
       const float nm = fmaxf(m, cm);
       float acc = s * exp2f(m - nm);
@@ -312,14 +339,21 @@ struct EpiGrad {
 #pragma unroll
         for (int i = 0; i < 32; ++i) q[i] = (gcol0 + i == y) ? 1.f : 0.f;
       }
-      load_bias32(p.bias, gcol0, p.V, bv);
       tmem_ld32(taddr + c * 32, z);
+      if (p.bias != nullptr) {  // warp-uniform
+        load_bias32(p.bias, gcol0, p.V, bv);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool ok = (gcol0 + i) < p.V;
-        const float t = (z[i] + bv[i]) * p.t_scale;
-        const float gv = cS * exp2f(t - lse2) - cQ * q[i];
-        z[i] = ok ? gv : 0.f;
+        for (int i = 0; i < 32; ++i) z[i] += bv[i];
+      }
+      if (gcol0 + 32 <= p.V) {  // warp-uniform: no column past V
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] = cS * exp2f(z[i] * p.t_scale - lse2) - cQ * q[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float gv = cS * exp2f(z[i] * p.t_scale - lse2) - cQ * q[i];
+          z[i] = (gcol0 + i) < p.V ? gv : 0.f;
+        }
       }
       if (rv) {
         // this row's 32 gradients of the chunk: two full 32-byte sectors
@@ -342,6 +376,126 @@ struct EpiGrad {
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) qa[j] = qb[j];
+    }
+  }
+};
+
+// Fused linear Jensen-Shannon divergence, student side of one vocabulary
+// chunk.  With the student probability p = 2^(t - lse2) (t = (acc + b) *
+// log2(e)/T, rounded to bf16 as the teacher's is), the teacher probability q
+// of the same entry (staged in bf16 by
+// an earlier teacher pass, chunk-relative rows of `ldg`) and m = beta p +
+// (1 - beta) q:
+//   loss mode (grad == 0): per (row, 128-column group) partial sums
+//       part[0][g][row] = sum p ln(p/m),
+//       part[1][g][row] = beta sum p ln(p/m) + (1 - beta) sum q ln(q/m);
+//   gradient mode (grad == 1): G = rowscale * beta * p * (ln(p/m) - K[row])
+//       as bf16 into the staging block, with per 32-row column sums for db.
+//       G may overwrite the teacher block itself: each thread reads the q of
+//       a 32-column chunk (coherent loads) before it stores that chunk's G.
+// 0 ln 0 is taken as 0.
+struct EpiJsd {
+  struct Params {
+    const __nv_bfloat16* bias;  // may be null
+    int BT, V;
+    int c0;          // first vocabulary column of the chunk
+    int ldg;         // row pitch (elements) of the staged teacher block and of G
+    const __nv_bfloat16* Qs;  // teacher probabilities of the chunk
+    float t_scale;
+    const float* lse2;   // [BT] student log2-sum-exp2
+    float beta;
+    int grad;
+    float* part;         // loss mode: [2][n_groups][BT]
+    long long part_plane;
+    __nv_bfloat16* G;    // gradient mode (may be Qs)
+    const float* K;      // [BT] KL(P || M) per row
+    const float* rowscale;  // [BT] 1 / (T D), 0 on dropped rows
+    float* dbpart;       // [row groups of 32][V] or null
+  };
+  __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
+                                                  int lane) {
+    const int row = row0 + quad * 32 + lane;
+    if (row < p.BT && p.c0 + n0 < p.V) {
+      const __nv_bfloat16* q = p.Qs + static_cast<size_t>(row) * p.ldg + n0;
+      prefetch_l2(q);
+      prefetch_l2(q + 64);
+    }
+  }
+  __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
+                                             int quad, int lane) {
+    const int row = row0 + quad * 32 + lane;
+    const bool rv = row < p.BT;
+    if (p.c0 + n0 >= p.V) return;  // warp-uniform
+    const __nv_bfloat16* qrow = p.Qs + static_cast<size_t>(rv ? row : 0) * p.ldg;
+    const float lse2 = rv ? p.lse2[row] : 0.f;
+    const float LN2 = 0.693147180559945309f;
+    const float beta = p.beta, omb = 1.f - p.beta;
+    const float gk = (p.grad && rv) ? p.K[row] : 0.f;
+    const float gs = (p.grad && rv) ? p.rowscale[row] * beta : 0.f;
+    float kp = 0.f, kq = 0.f;
+    uint4 qa[4], qb[4];
+    load_chunk32_rw(qrow, rv, n0, p.ldg, qa);
+#pragma unroll 1
+    for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
+      const int col0 = n0 + c * 32;
+      const int gcol0 = p.c0 + col0;
+      if (gcol0 >= p.V) break;  // warp-uniform
+      float q[32], bv[32], z[32];
+      if (c + 1 < TC_EPI_COLS / 32) load_chunk32_rw(qrow, rv, col0 + 32, p.ldg, qb);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+      tmem_ld32(taddr + c * 32, z);
+      if (p.bias != nullptr) {  // warp-uniform
+        load_bias32(p.bias, gcol0, p.V, bv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) z[i] += bv[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const bool ok = (gcol0 + i) < p.V;
+        // p rounded to bf16 like the staged teacher q, so that a teacher equal
+        // to the student gives p == q exactly (divergence and gradient 0)
+        const float pv = ok ? __bfloat162float(__float2bfloat16_rn(exp2f(z[i] * p.t_scale - lse2)))
+                            : 0.f;
+        const float qv = ok ? q[i] : 0.f;
+        const float mv = beta * pv + omb * qv;
+        const float lm = __log2f(mv);
+        // p ln(p/m) and q ln(q/m), 0 when the probability is 0
+        const float lp = pv > 0.f ? (__log2f(pv) - lm) * LN2 : 0.f;
+        if (!p.grad) {
+          kp = fmaf(pv, lp, kp);
+          kq += qv > 0.f ? qv * ((__log2f(qv) - lm) * LN2) : 0.f;
+        } else {
+          z[i] = pv > 0.f ? gs * pv * (lp - gk) : 0.f;
+        }
+      }
+      if (p.grad) {
+        if (rv) {
+          uint4* dst = reinterpret_cast<uint4*>(p.G + static_cast<size_t>(row) * p.ldg + col0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint4 u;
+            u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
+            u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
+            u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
+            u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
+            dst[j] = u;
+          }
+        }
+        if (p.dbpart != nullptr) {
+          const float colsum = warp_transpose_sum32(z, lane);
+          const int gc = gcol0 + lane;
+          if (gc < p.V)
+            p.dbpart[static_cast<size_t>(row0 / 32 + quad) * p.V + gc] = colsum;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) qa[j] = qb[j];
+    }
+    if (!p.grad && rv) {
+      const size_t o = static_cast<size_t>((p.c0 + n0) / TC_EPI_COLS) * p.BT + row;
+      p.part[o] = kp;
+      p.part[o + p.part_plane] = beta * kp + omb * kq;
     }
   }
 };
@@ -468,7 +622,8 @@ enum TcKind : int {
   KIND_STATS = 0,  // z tile -> softmax/KL statistics      A = X (K-major), B = W (K-major)
   KIND_GRAD = 1,   // z tile -> G staging (+ db partials)   A = X (K-major), B = W (K-major)
   KIND_DW = 2,     // dW rows = G^T X                       A = G (MN-major), B = X (MN-major)
-  KIND_DX = 3      // dX (+)= G W                           A = G (K-major), B = W (MN-major)
+  KIND_DX = 3,     // dX (+)= G W                           A = G (K-major), B = W (MN-major)
+  KIND_JSD = 4     // student z tile -> JSD partials / G     A = X (K-major), B = W (K-major)
 };
 __host__ __device__ constexpr bool kind_a_mn(int k) { return k == KIND_DW; }
 __host__ __device__ constexpr bool kind_b_mn(int k) { return k == KIND_DW || k == KIND_DX; }
@@ -503,6 +658,7 @@ struct TcLaunch {
   EpiGrad::Params grad;
   EpiStoreRows::Params dw;
   EpiAccumRows::Params dx;
+  EpiJsd::Params jsd;
 };
 
 // Problem and local tile index of sequence position t.  Problem 0 occupies
@@ -552,6 +708,7 @@ __device__ __forceinline__ void dispatch_epilogue(const TcLaunch& L, int kind, F
     case KIND_STATS: f(EpiStats{}, L.stats); break;
     case KIND_GRAD: f(EpiGrad{}, L.grad); break;
     case KIND_DW: f(EpiStoreRows{}, L.dw); break;
+    case KIND_JSD: f(EpiJsd{}, L.jsd); break;
     default: f(EpiAccumRows{}, L.dx); break;
   }
 }
