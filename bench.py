@@ -638,6 +638,7 @@ def run_ours(args):
             "kernels": kinds, "breakdown_check": breakdown_check,
             "gpu_launches": int((launches_per_step + (1 if args.dp else 0)) * args.steps),
             "clocks": clk, "sm_clock_in_kernel_mhz": sm_clock,
+            "gemm_ctas": pkg.flkl_gemm_ctas(),
             "other_workloads": others, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

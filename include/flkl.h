@@ -421,6 +421,11 @@ FLKL_API flkl_status flkl_wait_selftest(int* status_out, unsigned int limit_ms, 
 FLKL_API flkl_status flkl_clock_trace(uint64_t* out, int n_samples, unsigned int interval_ns,
                                       void* stream);
 
+/* SMs (CTAs, one per SM) that every GEMM launch of the library's tensor-core
+ * kernel occupies on the current device: as many CTA pairs (clusters of two)
+ * as are resident at once, times two; 0 without a usable device. */
+FLKL_API int flkl_gemm_ctas(void);
+
 /* Static text for a status code. */
 FLKL_API const char* flkl_status_string(int status);
 

@@ -26,7 +26,7 @@ __all__ = [
     "flkl_ce_forward_backward_dp", "count_valid", "flkl_selective_logprob_forward",
     "flkl_selective_logprob_backward", "selective_logprob", "SelectiveLogProb",
     "flkl_jsd_workspace_size", "flkl_jsd_forward_backward", "jsd_forward_backward",
-    "FusedLinearJSDLoss", "flkl_scale_cast", "flkl_clock_trace", "flkl_vocab_chunks",
+    "FusedLinearJSDLoss", "flkl_scale_cast", "flkl_clock_trace", "flkl_gemm_ctas", "flkl_vocab_chunks",
     "flkl_forward_backward_dp_events", "flkl_ce_forward_backward_dp_events",
 ]
 
@@ -112,6 +112,8 @@ def _lib():
         lib.flkl_scale_cast.restype = c.c_int
         lib.flkl_scale_cast.argtypes = [c.c_void_p, c.c_int, c.c_void_p, c.c_int, c.c_int64,
                                         c.c_void_p, c.c_void_p]
+        lib.flkl_gemm_ctas.restype = c.c_int
+        lib.flkl_gemm_ctas.argtypes = []
         lib.flkl_clock_trace.restype = c.c_int
         lib.flkl_clock_trace.argtypes = [c.c_void_p, c.c_int, c.c_uint, c.c_void_p]
         lib.flkl_vocab_chunks.restype = c.c_int
@@ -324,6 +326,10 @@ def flkl_forward_backward_profiled(X, W, b, Q, shift_labels, ignore_index, BT, H
 def flkl_scale_cast(src, src_dtype, dst, dst_dtype, n, scale, stream=None) -> int:
     return _lib().flkl_scale_cast(src, int(src_dtype), dst, int(dst_dtype), int(n), scale,
                                   stream)
+
+
+def flkl_gemm_ctas() -> int:
+    return _lib().flkl_gemm_ctas()
 
 
 def flkl_clock_trace(out_ptr, n_samples, interval_ns, stream=None) -> int:

@@ -170,19 +170,49 @@ bool make_blocked_map(CUtensorMap* m, const void* base, uint64_t blocked_extent,
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_group(const TcMaps& maps, const TcLaunch& L, cudaStream_t st) {
-  static bool attr_done[kMaxDevices] = {};
+// CTA pairs (clusters of 2) of the GEMM kernel that are resident at once on
+// the device, one CTA per SM (a cluster sits inside one GPC), cached per
+// device; 0 without a usable device.
+int g_tc_pairs[kMaxDevices] = {};
+
+int tc_pairs() {
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < kMaxDevices && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc_group_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = true;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  int pairs = cached ? g_tc_pairs[dev] : 0;
+  if (pairs == 0) {
+    if (cudaFuncSetAttribute(tc_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             TC_SMEM_BYTES) != cudaSuccess)
+      return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = TC_SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, tc_group_kernel, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();  // clear a failed query; fall back to the SM count
+      n = num_sms() / 2;
+    }
+    pairs = std::max(1, std::min(n, num_sms() / 2));
+    if (cached) g_tc_pairs[dev] = pairs;
   }
+  return pairs;
+}
+
+cudaError_t launch_group(const TcMaps& maps, const TcLaunch& L, cudaStream_t st) {
+  const int pairs = tc_pairs();
+  if (pairs == 0) return cudaErrorInvalidDevice;
   if (L.total_tiles <= 0) return cudaSuccess;
-  // one CTA pair (cluster of 2) per claimed tile, at most one CTA per SM
-  const int grid = 2 * static_cast<int>(std::min<long long>(L.total_tiles, num_sms() / 2));
+  // one CTA pair (cluster of 2) per claimed tile, at most the pairs that are
+  // resident at once (persistent)
+  const int grid = 2 * static_cast<int>(std::min<long long>(L.total_tiles, pairs));
   tc_group_kernel<<<grid, TC_THREADS, TC_SMEM_BYTES, st>>>(maps, L);
   return cudaGetLastError();
 }
@@ -1213,6 +1243,8 @@ flkl_status flkl_ce_forward_backward_dp(const void* X, const void* W, const void
                                loss, dX, dW, db, workspace, workspace_bytes, stream, nullptr,
                                BT > 0 ? target : nullptr, n_valid_total);
 }
+
+int flkl_gemm_ctas(void) { return 2 * tc_pairs(); }
 
 int flkl_vocab_chunks(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW,
                       int compute_db, int64_t* bounds, int capacity) {

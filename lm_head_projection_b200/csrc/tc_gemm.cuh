@@ -874,9 +874,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         // Descriptors of this tile: a constant upper word (SBO, version,
         // swizzle) and a lower word (LBO | start address >> 4) that only moves
         // by fixed steps between K slices and stages (see stage_desc).
+        // (the start-address field holds bits [4, 18) of the CTA's shared
+        // address; a shared address may carry the CTA's rank above them)
         const DescSteps da = desc_steps(a_mn), db = desc_steps(b_mn);
-        const uint32_t a_lo0 = da.lo_base + (smem_u32(sA) >> 4);
-        const uint32_t b_lo0 = db.lo_base + (smem_u32(sB) >> 4);
+        const uint32_t a_lo0 = da.lo_base + ((smem_u32(sA) & 0x3FFFFu) >> 4);
+        const uint32_t b_lo0 = db.lo_base + ((smem_u32(sB) & 0x3FFFFu) >> 4);
         for (int kb = 0; kb < P.num_kb; ++kb) {
           if (!mbar_wait(&full[stage], phase, wc)) {
             ok = false;
