@@ -34,6 +34,7 @@ unsigned long long g_wait_limit_ns = 4000ull * 1000000ull;
 namespace {
 
 constexpr size_t kStagingBudget = size_t(256) << 20;  // bytes of G staging at most
+constexpr long long kPairsPerWave = 74;               // CTA pairs of a 148-SM part
 constexpr int kMaxDevices = 64;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -65,9 +66,23 @@ bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int 
   p.m_tiles = cdiv(BT, p.tile_m);
   p.n_tiles = cdiv(V, p.tile_n);
   p.n_stat = p.tc ? cdiv(V, TC_EPI_COLS) : p.n_tiles;
-  // Chunk width: at most V/8 (rounded up to the tile width) and at most the
-  // staging budget; never below one tile.
+  // Chunk width: about V/8 (rounded up to the tile width) and at most the
+  // staging budget; never below one tile.  On the tensor-core path, when one
+  // chunk's pass-2 tiles make only a few waves, the width grows (by at most a
+  // half) until they fill whole waves of the CTA pairs of a 148-SM part: the
+  // first chunk's pass 2 runs in a launch of its own.
   long long vc = cdiv(cdiv(V, 8), p.tile_n) * p.tile_n;
+  if (p.tc && BT > 0) {
+    const long long nt0 = vc / p.tile_n;
+    if (p.m_tiles * nt0 < 4 * kPairsPerWave) {
+      for (long long nt = nt0; nt * 2 <= nt0 * 3; ++nt) {
+        if ((p.m_tiles * nt) % kPairsPerWave == 0) {
+          vc = nt * p.tile_n;
+          break;
+        }
+      }
+    }
+  }
   if (BT > 0) {
     long long cap = static_cast<long long>(kStagingBudget / (size_t(BT) * elem));
     cap = (cap / p.tile_n) * p.tile_n;
