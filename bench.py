@@ -606,8 +606,11 @@ def run_ours(args):
             and args.workload == HEADLINE):
         others = {}
         for name in OTHER_WORKLOADS:
-            others[name] = measure_other(pkg, ALL_WORKLOADS[name], dev, stream, args,
-                                         peaks, peaks_src, gpu_index)
+            try:
+                others[name] = measure_other(pkg, ALL_WORKLOADS[name], dev, stream, args,
+                                             peaks, peaks_src, gpu_index)
+            except Exception as exc:  # keep the headline line whatever happens here
+                others[name] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
             torch.cuda.empty_cache()
 
     cpu = None
