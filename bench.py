@@ -917,9 +917,10 @@ def run_logprob(args):
         "config": {"workload": name, "BT": w.BT, "H": w.H, "V": w.V, "compute_dW": cw,
                    "compute_db": cb, "l2": "inputs larger than L2 (W), no flush"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
-                     "traffic": None, "scope": "whole step (counted FLOPs)",
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "traffic": None, "scope": "whole step (counted FLOPs), burst peak",
                      "peak_source": peak_src},
         "cpu_baseline": {"value": round(rows / t_cpu, 2), "unit": "tokens/s",
                          "cores": host_threads(), "kind": "oracle",
@@ -997,11 +998,13 @@ def run_jsd(args):
                    "Ht": w.H, "V": w.V, "beta": beta, "compute_dW": True,
                    "l2": "inputs larger than L2 (W, Wt), no flush"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
-                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "traffic": None,
                      "scope": "whole call; counted = teacher + student logits, dX, dW "
-                              "(8 GEMMs of that size run)", "peak_source": peak_src},
+                              "(8 GEMMs of that size run); burst peak",
+                     "peak_source": peak_src},
         "cpu_baseline": {"value": round(rows / t_cpu, 2), "unit": "tokens/s",
                          "cores": host_threads(), "kind": "oracle",
                          "sample": f"{rows} rows, fp64 numpy, {t_cpu:.1f} s"},
