@@ -175,14 +175,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
-// Bring a 2-D tile into L2 only (no shared memory, no completion signal).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 // 2-D tiled load issued by either CTA of a pair into its own shared memory,
 // with completion signalled on an mbarrier that may live in the peer CTA
 // (`bar_cluster` is a cluster-window address).  No multicast.

@@ -46,12 +46,11 @@ constexpr int TC_BK = FLKL_TC_BK;     // K depth of a ring stage (a multiple of 
 constexpr int TC_KSUB = TC_BK / 64;   // 128-byte swizzle atoms along K per stage
 constexpr int TC_STAGES = FLKL_TC_STAGES;
 static_assert(TC_BK % 64 == 0 && TC_BK <= 256, "stage depth: a multiple of 64, at most 256");
-constexpr int TC_PREFETCH_KB = 0;     // L2 prefetch distance of the producer, in k-blocks
 constexpr int TC_EPI_WARPS = 8;       // two per TMEM lane quarter
 constexpr int TC_EPI_COLS = 128;      // accumulator columns per epilogue warp
 constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
-constexpr int TC_A_BYTES = TC_HM * TC_BK * 2;  // 16 KiB: this CTA's A rows
-constexpr int TC_B_BYTES = TC_HM * TC_BK * 2;  // 16 KiB: this CTA's half of B
+constexpr int TC_A_BYTES = TC_HM * TC_BK * 2;  // this CTA's A rows (32 KiB at TC_BK = 128)
+constexpr int TC_B_BYTES = TC_HM * TC_BK * 2;  // this CTA's half of B (32 KiB at TC_BK = 128)
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + TC_B_BYTES;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 256 + 1024;
@@ -78,18 +77,6 @@ __device__ __forceinline__ void tma_half_stage(const CUtensorMap* map, bool mn_m
   } else {
     tma_load_2d_pair(map, bar_cluster, dst, mn0, k0);
     tma_load_2d_pair(map, bar_cluster, dst + TC_BK * 128, mn0 + 64, k0);
-  }
-}
-
-// L2 prefetch of the same boxes tma_half_stage would load.
-__device__ __forceinline__ void prefetch_half_stage(const CUtensorMap* map, bool mn_major, int mn0,
-                                                    int k0) {
-  if (!mn_major) {
-#pragma unroll
-    for (int s = 0; s < TC_KSUB; ++s) tma_prefetch_l2_2d(map, k0 + 64 * s, mn0);
-  } else {
-    tma_prefetch_l2_2d(map, mn0, k0);
-    tma_prefetch_l2_2d(map, mn0 + 64, k0);
   }
 }
 
@@ -821,12 +808,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                          kb * TC_BK + P.a_k_off);
           tma_half_stage(mB, b_mn, P.b_blocked, fbar, sB + stage * TC_B_BYTES, n0,
                          kb * TC_BK + P.b_k_off);
-          if (TC_PREFETCH_KB > 0 && kb + TC_PREFETCH_KB < P.num_kb) {
-            // keep the L2 a few k-blocks ahead of the copies (HBM misses become L2 hits)
-            const int kp = (kb + TC_PREFETCH_KB) * TC_BK;
-            prefetch_half_stage(mA, a_mn, m0, kp + P.a_k_off);
-            prefetch_half_stage(mB, b_mn, n0, kp + P.b_k_off);
-          }
           ++issued;
           if (++stage == TC_STAGES) {
             stage = 0;
