@@ -34,6 +34,7 @@ unsigned long long g_wait_limit_ns = 4000ull * 1000000ull;
 namespace {
 
 constexpr size_t kStagingBudget = size_t(256) << 20;  // bytes of G staging at most
+constexpr size_t kLogitCacheBudget = size_t(256) << 20;  // bytes of the chunk-0 logits cache at most
 constexpr long long kPairsPerWave = 74;               // CTA pairs of a 148-SM part
 constexpr int kMaxDevices = 64;
 
@@ -49,7 +50,8 @@ struct Plan {
   long long db_groups;
   long long n_counters;  // tile counters of the persistent launches, then combine tickets
   long long comb_rowblocks, comb_splits;  // grid of k_combine_split
-  size_t off_cnt, off_st, off_rows, off_cpart, off_G, off_dx, off_db, total;
+  long long zc_cols;     // columns of the first chunk whose logits pass 1 keeps (0: none)
+  size_t off_cnt, off_st, off_rows, off_cpart, off_G, off_zc, off_dx, off_db, total;
   size_t g_stride;       // bytes between the two G staging buffers
 };
 
@@ -112,6 +114,16 @@ bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int 
   // is produced while chunk c's is consumed
   p.g_stride = align256(size_t(BT) * vc * elem);
   off += p.g_stride * ((p.tc && p.nchunks > 1) ? 2 : 1);
+  // tensor-core path: pass 1 keeps the fp32 logits of the first chunk
+  // (32-row blocks), as many of its columns as the budget holds (a multiple
+  // of the tile width), so that pass 2 needs no GEMM for them
+  const size_t rows32 = size_t(cdiv(BT, 32)) * 32;
+  p.zc_cols = 0;
+  if (p.tc && BT > 0)
+    p.zc_cols = std::min<long long>(
+        vc, static_cast<long long>(kLogitCacheBudget / (rows32 * 4)) / p.tile_n * p.tile_n);
+  p.off_zc = off;
+  if (p.zc_cols > 0) off += align256(rows32 * size_t(p.zc_cols) * 4);
   p.off_dx = off;
   if (p.nchunks > 1) off += align256(size_t(BT) * H * 4);
   p.off_db = off;
@@ -404,26 +416,36 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     L.err_flag = &ctl->err;
     L.wait_limit_ns = g_wait_limit_ns;
     L.stats = EpiStats::Params{Q, b, BT, V, t_scale, eps, stats,
-                               static_cast<long long>(P.n_stat) * BT, target};
+                               static_cast<long long>(P.n_stat) * BT, target, nullptr, 0};
     return L;
   };
   auto chunk_c0 = [&](long long c) { return static_cast<int>(c * P.Vc); };
   auto chunk_w = [&](long long c) {
     return static_cast<int>(std::min<long long>(P.Vc, V - c * P.Vc));
   };
+  auto grad_params = [&](long long c) {
+    return EpiGrad::Params{Q,       b,    BT,    V,     chunk_c0(c), ldg,   Gbuf[c & 1],
+                           t_scale, lse2, coefS, coefQ, dbpart,      target};
+  };
   // pass-2 problem of chunk c: logits of the chunk again -> G staging
   auto add_grad = [&](TcLaunch& L, TcMaps& maps, long long c) {
-    const int c0 = chunk_c0(c);
-    L.grad = EpiGrad::Params{Q,     b,     BT,    V,     c0,     ldg,   Gbuf[c & 1],
-                             t_scale, lse2, coefS, coefQ, dbpart, target};
-    return add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, c0, 0);
+    L.grad = grad_params(c);
+    return add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, chunk_c0(c), 0);
   };
+  // a whole call keeps the first chunk's logits from pass 1 (when the cache
+  // fits); the forward-only and backward-only calls recompute them
+  float* zc = reinterpret_cast<float*>(ws + P.off_zc);
+  const bool cached = ph.forward && ph.backward && ph.dlogp == nullptr && P.zc_cols > 0;
 
   if (ph.forward) {
     // pass 1: statistics over all V
     {
       TcLaunch L = new_launch(0);
       TcMaps maps{};
+      if (cached) {
+        L.stats.zc = zc;
+        L.stats.zc_cols = static_cast<int>(P.zc_cols);
+      }
       add_problem(L, maps, KIND_STATS, BT, V, H, 1, mX_k, mW_k);
       Rec r_(rec, 1, 2.0 * BT * static_cast<double>(V) * H);
       FLKL_CUDA(launch_group(maps, L, st));
@@ -433,8 +455,30 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
   }
   if (!ph.backward) return FLKL_OK;
   FLKL_CUDA(upstream_coefs(ph.dlogp, target, BT, ignore_index, V, T, coefS, coefQ, st, rec));
-  // pass 2 of chunk 0 alone
-  {
+  if (cached) {
+    // pass 2 of chunk 0 from the logits cache
+    {
+      Rec r_(rec, 4);
+      const long long warps = cdiv(BT, 32) * (P.zc_cols / 32);
+      k_grad_cached<<<static_cast<unsigned>(cdiv(warps, 8)), 256, 0, st>>>(
+          grad_params(0), zc, static_cast<int>(P.zc_cols));
+      FLKL_CUDA(cudaGetLastError());
+    }
+    // the chunk's columns past the cache, if any: pass 2 as a GEMM
+    const long long rest = chunk_w(0) - P.zc_cols;
+    if (rest > 0) {
+      TcLaunch L = new_launch(1);
+      TcMaps maps{};
+      L.grad = grad_params(0);
+      L.grad.c0 = static_cast<int>(P.zc_cols);
+      L.grad.G = Gbuf[0] + P.zc_cols;
+      add_problem(L, maps, KIND_GRAD, BT, rest, H, 1, mX_k, mW_k, 0, static_cast<int>(P.zc_cols),
+                  0);
+      Rec r_(rec, 4, 2.0 * BT * static_cast<double>(rest) * H);
+      FLKL_CUDA(launch_group(maps, L, st));
+    }
+  } else {
+    // pass 2 of chunk 0 alone
     TcLaunch L = new_launch(1);
     TcMaps maps{};
     add_grad(L, maps, 0);
@@ -471,9 +515,12 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
     ph.chunk_finished(c, st);
   }
   if (compute_db) {
+    // the 32-row groups that hold rows (k_grad_cached writes no partials for
+    // the all-padding groups of the last row tile; the GEMM epilogues write
+    // zeros there)
     Rec r_(rec, 7);
     k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
-        dbpart, static_cast<int>(P.db_groups), V, db, accum_fp32);
+        dbpart, static_cast<int>(cdiv(BT, 32)), V, db, accum_fp32);
     FLKL_CUDA(cudaGetLastError());
   }
   return FLKL_OK;

@@ -167,6 +167,13 @@ struct EpiStats {
     float* st;      // [5][n_groups][BT], n_groups = ceil(V/128)
     long long st_plane;  // n_groups * BT
     const int64_t* target;  // cross-entropy mode: q = one-hot at target[row]; else null
+    // logits cache of the first vocabulary chunk (null: none): the raw
+    // accumulators of columns [0, zc_cols) in 32 x 32 blocks, block
+    // (row / 32, column / 32) at ((row / 32) * (zc_cols / 32) + column / 32) * 1024,
+    // element (column % 32) * 32 + row % 32, so that a warp (lane = row) stores
+    // and reads each column of a block as one 128-byte line
+    float* zc;
+    int zc_cols;
   };
   __device__ __forceinline__ static void prefetch(const Params& p, int row0, int n0, int quad,
                                                   int lane) {
@@ -204,6 +211,12 @@ struct EpiStats {
         for (int i = 0; i < 32; ++i) q[i] = (col0 + i == y) ? 1.f : 0.f;
       }
       tmem_ld32(taddr + c * 32, z);
+      if (p.zc != nullptr && col0 < p.zc_cols && rv) {  // (the first condition is warp-uniform)
+        float* dst = p.zc +
+                     (static_cast<size_t>(row >> 5) * (p.zc_cols >> 5) + (col0 >> 5)) * 1024 + lane;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[i * 32] = z[i];
+      }
       if (p.bias != nullptr) {  // warp-uniform
         load_bias32(p.bias, col0, p.V, bv);
 #pragma unroll
@@ -298,6 +311,56 @@ struct EpiGrad {
       if (gc + 64 < p.V) prefetch_l2(q + 64);
     }
   }
+  // One gradient value from the logit z (bias added): (S p - q) / (T D) with
+  // p = 2^(z log2(e) / T - lse2).  Both multiply-adds are explicit so that
+  // every caller rounds the same way.
+  __device__ __forceinline__ static float value(float z, float t_scale, float lse2, float cS,
+                                                float cQ, float q) {
+    return __fmaf_rn(cS, exp2f(__fmaf_rn(z, t_scale, -lse2)), -(cQ * q));
+  }
+  // The gradients of 32 columns of one row (lane = row of a 32-row group)
+  // from their logits z (the accumulator, before the bias): bf16 into the
+  // staging row and, with db, the group's column sums.  Shared by the
+  // epilogue and k_grad_cached, which therefore give the same bits.
+  __device__ __forceinline__ static void cols32(const Params& p, float (&z)[32],
+                                                const float (&q)[32], int row, bool rv,
+                                                int rgroup, int col0, int gcol0, float lse2,
+                                                float cS, float cQ, int lane) {
+    if (p.bias != nullptr) {  // warp-uniform
+      float bv[32];
+      load_bias32(p.bias, gcol0, p.V, bv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] += bv[i];
+    }
+    if (gcol0 + 32 <= p.V) {  // warp-uniform: no column past V
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] = value(z[i], p.t_scale, lse2, cS, cQ, q[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float gv = value(z[i], p.t_scale, lse2, cS, cQ, q[i]);
+        z[i] = (gcol0 + i) < p.V ? gv : 0.f;
+      }
+    }
+    if (rv) {
+      // this row's 32 gradients of the chunk: two full 32-byte sectors
+      uint4* dst = reinterpret_cast<uint4*>(p.G + static_cast<size_t>(row) * p.ldg + col0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 u;
+        u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
+        u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
+        u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
+        u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
+        dst[j] = u;
+      }
+    }
+    if (p.dbpart != nullptr) {
+      const float colsum = warp_transpose_sum32(z, lane);
+      const int gc = gcol0 + lane;
+      if (gc < p.V) p.dbpart[static_cast<size_t>(rgroup) * p.V + gc] = colsum;
+    }
+  }
   __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
                                              int quad, int lane) {
     const int row = row0 + quad * 32 + lane;
@@ -317,7 +380,7 @@ struct EpiGrad {
       const int col0 = n0 + c * 32;
       const int gcol0 = p.c0 + col0;
       if (gcol0 >= p.V) break;  // warp-uniform
-      float q[32], bv[32], z[32];
+      float q[32], z[32];
       if (!ce) {
         if (c + 1 < TC_EPI_COLS / 32) load_chunk32(qrow, rv, gcol0 + 32, p.V, qb);
 #pragma unroll
@@ -327,40 +390,7 @@ struct EpiGrad {
         for (int i = 0; i < 32; ++i) q[i] = (gcol0 + i == y) ? 1.f : 0.f;
       }
       tmem_ld32(taddr + c * 32, z);
-      if (p.bias != nullptr) {  // warp-uniform
-        load_bias32(p.bias, gcol0, p.V, bv);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] += bv[i];
-      }
-      if (gcol0 + 32 <= p.V) {  // warp-uniform: no column past V
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] = cS * exp2f(z[i] * p.t_scale - lse2) - cQ * q[i];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float gv = cS * exp2f(z[i] * p.t_scale - lse2) - cQ * q[i];
-          z[i] = (gcol0 + i) < p.V ? gv : 0.f;
-        }
-      }
-      if (rv) {
-        // this row's 32 gradients of the chunk: two full 32-byte sectors
-        uint4* dst = reinterpret_cast<uint4*>(p.G + static_cast<size_t>(row) * p.ldg + col0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 u;
-          u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
-          u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
-          u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
-          u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
-          dst[j] = u;
-        }
-      }
-      if (p.dbpart != nullptr) {
-        const float colsum = warp_transpose_sum32(z, lane);
-        const int gc = gcol0 + lane;
-        if (gc < p.V)
-          p.dbpart[static_cast<size_t>(row0 / 32 + quad) * p.V + gc] = colsum;
-      }
+      cols32(p, z, q, row, rv, row0 / 32 + quad, col0, gcol0, lse2, cS, cQ, lane);
 #pragma unroll
       for (int j = 0; j < 4; ++j) qa[j] = qb[j];
     }
@@ -494,6 +524,42 @@ struct EpiJsd {
 // warp store of 8-byte pairs writes 8 rows x 32 bytes (whole sectors).
 
 // dW rows of one chunk: out[c0 + m][n] = acc, fp32 or bf16.
+// Pass 2 of the first vocabulary chunk from the logits cache that pass 1
+// filled (EpiStats::Params::zc): the same accumulators pass 2 would compute
+// again (same operands, same K order), so the same gradients, without the
+// GEMM.  One warp per 32 rows x 32 columns, lane = row; 8 warps per block.
+__global__ void __launch_bounds__(256) k_grad_cached(const EpiGrad::Params p,
+                                                     const float* __restrict__ zc, int zc_cols) {
+  const int lane = threadIdx.x & 31;
+  const int ncc = zc_cols >> 5;
+  const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (w >= static_cast<long long>((p.BT + 31) >> 5) * ncc) return;  // warp-uniform
+  const int rg = static_cast<int>(w / ncc), col0 = static_cast<int>(w % ncc) * 32;
+  const int gcol0 = p.c0 + col0;
+  if (gcol0 >= p.V) return;  // warp-uniform
+  const int row = rg * 32 + lane;
+  const bool rv = row < p.BT;
+  float z[32], q[32];
+  const float* src = zc + static_cast<size_t>(w) * 1024 + lane;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) z[i] = rv ? src[i * 32] : 0.f;
+  if (p.Q != nullptr) {  // warp-uniform
+    uint4 qa[4];
+    load_chunk32(p.Q + static_cast<size_t>(rv ? row : 0) * p.V, rv, gcol0, p.V, qa);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+  } else {
+    long long y = rv ? p.target[row] : -1;
+    if (y >= p.V) y = -1;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) q[i] = (gcol0 + i == y) ? 1.f : 0.f;
+  }
+  const float lse2 = rv ? p.lse2[row] : 0.f;
+  const float cS = rv ? p.coefS[row] : 0.f;
+  const float cQ = rv ? p.coefQ[row] : 0.f;
+  EpiGrad::cols32(p, z, q, row, rv, rg, col0, gcol0, lse2, cS, cQ, lane);
+}
+
 struct EpiStoreRows {
   struct Params {
     void* out;

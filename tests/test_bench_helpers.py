@@ -123,6 +123,10 @@ def test_step_roofline_cap_and_fractions():
     r = bench.step_roofline(w, ms, peaks, "measured")
     assert r["frac_of_burst"] == pytest.approx(0.5, abs=1e-4)
     assert r["cap_with_recompute"] == pytest.approx(2 / 3, abs=1e-4)
+    # with the executed GEMM FLOPs of a call (first chunk not recomputed)
+    executed = w.flops_counted() * 1.4
+    r = bench.step_roofline(w, ms, peaks, "measured", executed=executed)
+    assert r["cap_with_recompute"] == pytest.approx(1 / 1.4, abs=1e-4)
 
 
 def test_max_over_ranks_without_a_group_is_the_value():
