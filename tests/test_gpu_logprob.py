@@ -157,3 +157,25 @@ def test_unit_upstream_gradient_gives_the_cross_entropy_gradients():
     for k in ("dX", "dW", "db"):
         assert float((got[k] - ce[k]).abs().max()) <= 1e-6, k
     assert abs(float(-got["logp"].sum() / kept.sum()) - float(ce["loss"])) <= 1e-5
+
+
+def test_kept_first_chunk_gives_the_recomputed_gradients():
+    """A whole cross-entropy call (sum reduction) forms the first vocabulary
+    chunk's gradient block from the logits pass 1 kept; the selective
+    log-probability backward call with upstream gradient -1 per row forms
+    the same block by recomputing the logits.  Both are G = (p - onehot) / T
+    on the kept rows, so dX, dW and db agree bit for bit."""
+    import lm_head_projection_b200 as pkg
+
+    T = 1.3
+    inp, tgt, _ = _inputs("bf16", 300, 128, 4104, True, T, seed=21)
+    dev = torch.device("cuda:0")
+    X, W, b = inp["X"].to(dev), inp["W"].to(dev), inp["b"].to(dev)
+    bounds = pkg.flkl_vocab_chunks(300, 128, 4104, 1, True, True)
+    assert len(bounds) > 2  # several chunks: the first kept, the rest recomputed
+    whole = pkg.cross_entropy_forward_backward(X, W, b, tgt.to(dev), -100, T, "sum",
+                                               compute_dW=True, compute_db=True,
+                                               accum_fp32=True, check_status=True)
+    split = _gpu(pkg, inp, tgt, -torch.ones(300), "bf16", T, True, True)
+    for k in ("dX", "dW", "db"):
+        assert torch.equal(whole[k], split[k]), k
