@@ -61,15 +61,42 @@ def load_peaks():
 GEMM_SOURCES = ("flkl_api.cu", "ptx.cuh", "row_kernels.cuh", "tc_gemm.cuh")
 
 
+def code_only(src: str) -> str:
+    """C / CUDA source without its comments and blank space (string and
+    character literals kept as they are), so that editing a comment does not
+    count as a change of the code."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources the fused-loss kernels are built from."""
+    """Hash of the code (comments and blank space left out) of the CUDA
+    sources the fused-loss kernels are built from."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "lm_head_projection_b200", "csrc")
     for fn in GEMM_SOURCES:
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+            h.update(fn.encode() + b"\0" + code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -18,12 +18,13 @@
  *     S_r = sum_v q_rv,   dX = G W,   dW = G^T X,   db = sum_r G_r,
  *
  * and dW / db only when asked for (the frozen-head change of the GRPO page,
- * section Summary).  The BT x V logits are never written to device memory: the
- * library recomputes them tile by tile in two passes and stages only a
- * bounded BT x Vc block of G (Vc about V/8, rounded up to the tile width);
- * on the bf16 path pass 1 also keeps the fp32 logits of the first chunk (at
- * most 256 MiB), from which the first chunk's pass 2 forms G without a
- * GEMM.
+ * section Summary).  The BT x V logits are never written to device memory as
+ * a whole: the library computes them tile by tile in two passes (statistics,
+ * then the gradient per vocabulary chunk, recomputing the logits) and stages
+ * only a bounded BT x Vc block of G (Vc about V/8, rounded up to the tile
+ * width); on the bf16 path pass 1 keeps the fp32 logits of the first chunk
+ * only (at most 256 MiB), from which that chunk's G is formed without a
+ * second GEMM.
  *
  * Declared below, besides that call: the same path with a one-hot teacher
  * (cross-entropy) and as per-token log-probabilities with a separate backward

@@ -2,17 +2,24 @@
 // the pass plan and workspace layout, TMA tensor maps, and the launch
 // sequence on the caller's stream.
 //
-// Launch sequence of one call (bf16):
-//   k_prepare        N_valid, divisor D, 1/(T D); clears the status word
-//   pass 1  (tc)     z tiles = X W^T in TMEM, fused softmax/KL statistics
-//   k_combine        per-row lse and row loss, gradient coefficients
-//   k_loss           loss = sum of row losses / D (fixed order)
-//   per vocabulary chunk c of width Vc:
-//     pass 2 (tc)    z tiles of the chunk again, G = (S p - q)/(T D) -> bf16
-//                    staging [BT x Vc], db column partials
-//     dW gemm (tc)   dW[c] = G_c^T X (only when dW is asked for)
-//     dX gemm (tc)   dX (+)= G_c W[c] (fp32 partial across chunks)
+// Launch sequence of one whole call (bf16):
+//   k_prepare        N_valid, divisor D, 1/(T D); clears the status word and
+//                    the tile counters
+//   pass 1 (tc)      z tiles = X W^T in TMEM, fused softmax/KL statistics per
+//                    (row, 128-column group); the first chunk's raw logits
+//                    kept (fp32, up to a budget)
+//   k_combine_split  per-row lse and row loss, gradient coefficients, and the
+//                    loss = sum of row losses / D (fixed order)
+//   k_grad_cached    pass 2 of chunk 0 from the kept logits: G = (S p - q)/(T D)
+//                    -> bf16 staging [BT x Vc], db column partials (a pass-2
+//                    GEMM covers the chunk's columns past the budget)
+//   per vocabulary chunk c of width Vc, one grouped launch (tc):
+//                    dX(c): dX (+)= G_c W[c] (fp32 partial across chunks);
+//                    pass 2 of chunk c+1: its z tiles again -> G_{c+1};
+//                    dW(c) = G_c^T X (only when dW is asked for)
 //   k_db_reduce      db (only when asked for)
+// Forward-only and backward-only calls (selective log-probability) run pass
+// 1 and the merge, or pass 2 of every chunk by GEMM and the chunk launches.
 
 #include <cudaTypedefs.h>
 

@@ -9,9 +9,11 @@
 // of B; the even CTA issues the MMAs, which read A and B from both CTAs'
 // shared memory and write rows [128r, 128r+128) of D into CTA r's TMEM.
 //
-// Roles (6 warps per CTA, one CTA per SM):
-//   warp 0      TMA producer (both CTAs): a 6-deep ring of 32 KiB stages;
-//               every copy signals the even CTA's `full` barrier;
+// Roles (10 warps per CTA, one CTA per SM):
+//   warp 0      TMA producer (both CTAs): a ring of TC_STAGES stages of
+//               TC_BK-deep K blocks (3 x 64 KiB per CTA at the default
+//               TC_BK = 128); every copy signals the even CTA's `full`
+//               barrier;
 //   warp 1      TMEM owner (both CTAs, 512 columns = two 256-column fp32
 //               accumulators) and, in the even CTA, the MMA issuer;
 //               tcgen05.commit arrives on both CTAs' `empty` (stage free)
@@ -23,7 +25,9 @@
 //               even CTA's `tempty` barrier.
 //
 // Operands may be K-major (rows of K contiguous) or MN-major (K rows of M or N
-// contiguous); both are loaded by plain 2-D TMA tile copies, never multicast.
+// contiguous); both are loaded by plain TMA tile copies (one 3-D "blocked"
+// copy per operand and stage when the inner extent is a multiple of 64,
+// else 2-D copies), never multicast.
 // Every wait is bounded (see mbar_wait); on a timeout the CTA stops, drains
 // its own in-flight copies and MMAs, frees TMEM and returns.
 #pragma once

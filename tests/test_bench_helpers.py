@@ -43,6 +43,15 @@ def test_dram_traffic_lookup_follows_the_kernel_sources():
     assert bench.dram_traffic("no_such_workload", "chunk") is None
 
 
+def test_kernel_hash_ignores_comments_but_not_code():
+    src = ('int a = 1; // one\n/* two\n lines */ const char* s = "x // y /* z */";\n'
+           "char q = '\"';  int b = 2;\n")
+    assert bench.code_only(src) == ('int a = 1; const char* s = "x // y /* z */"; '
+                                    "char q = '\"'; int b = 2;")
+    assert bench.code_only(src.replace("// one", "// changed")) == bench.code_only(src)
+    assert bench.code_only(src.replace("b = 2", "b = 3")) != bench.code_only(src)
+
+
 def _sampler_with(tmp_path, lines, t0=None, t1=None):
     s = object.__new__(bench.ClockSampler)
     s.path = str(tmp_path / "clocks.csv")
