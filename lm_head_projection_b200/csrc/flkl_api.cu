@@ -514,7 +514,6 @@ flkl_status run_tc(const Plan& P, const __nv_bfloat16* X, const __nv_bfloat16* W
       // 1.7 % faster on the chunk launches than vocabulary blocks fastest)
       add_problem(L, maps, KIND_DW, Vw, H, BT, 0, mG_mn, mX_mn);
     }
-    L.mix = 0;  // problems in sequence (interleaving pass-2 and dW tiles measured slower)
     double f = 2.0 * BT * static_cast<double>(Vw) * H * (1 + (compute_dW ? 1 : 0));
     if (c + 1 < P.nchunks) f += 2.0 * BT * static_cast<double>(chunk_w(c + 1)) * H;
     {

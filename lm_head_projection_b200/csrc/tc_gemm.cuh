@@ -706,7 +706,6 @@ struct TcMaps {
 struct TcLaunch {
   int nprob;
   int total_tiles;
-  int mix;  // interleave problems 1 and 2 (see find_problem)
   TcProblem prob[TC_MAX_PROBLEMS];
   int* counter;  // tile counter of this launch, 0 at launch
   int* err_flag;
@@ -718,35 +717,13 @@ struct TcLaunch {
   EpiJsd::Params jsd;
 };
 
-// Problem and local tile index of sequence position t.  Problem 0 occupies
-// the first tiles; when L.mix is set, problems 1 and 2 are interleaved in
-// proportion to their tile counts over the rest of the sequence (so that
-// compute-heavy and store-heavy tiles run side by side), otherwise they
-// follow one another.
+// Problem and local tile index of sequence position t: the problems' tiles
+// follow one another in problem order.
 __device__ __forceinline__ int find_problem(const TcLaunch& L, int t, int& local) {
-  if (L.nprob == 1 || t < L.prob[1].tile_begin) {
-    local = t;
-    return 0;
-  }
-  const int j = t - L.prob[1].tile_begin;
-  if (L.mix && L.nprob == 3) {
-    const long long n1 = L.prob[1].m_tiles * static_cast<long long>(L.prob[1].n_tiles);
-    const long long n = L.total_tiles - L.prob[1].tile_begin;
-    const long long c_j = (static_cast<long long>(j) * n1) / n;        // problem-1 tiles before j
-    const long long c_j1 = (static_cast<long long>(j + 1) * n1) / n;
-    if (c_j1 > c_j) {
-      local = static_cast<int>(c_j);
-      return 1;
-    }
-    local = static_cast<int>(j - c_j);
-    return 2;
-  }
-  if (L.nprob == 3 && t >= L.prob[2].tile_begin) {
-    local = t - L.prob[2].tile_begin;
-    return 2;
-  }
-  local = j;
-  return 1;
+  int pi = 0;
+  while (pi + 1 < L.nprob && t >= L.prob[pi + 1].tile_begin) ++pi;
+  local = t - L.prob[pi].tile_begin;
+  return pi;
 }
 
 __device__ __forceinline__ void problem_tile(const TcProblem& P, int local, int& mb, int& nb) {
