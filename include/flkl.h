@@ -287,7 +287,8 @@ typedef enum {
   FLKL_LAUNCH_STATS = 1,    /* pass 1: logits GEMM + softmax/KL statistics    */
   FLKL_LAUNCH_COMBINE = 2,  /* per-row log-sum-exp and row loss              */
   FLKL_LAUNCH_LOSS = 3,     /* reduction of the row losses                   */
-  FLKL_LAUNCH_GRAD = 4,     /* pass 2 of one chunk: logits again + G staging */
+  FLKL_LAUNCH_GRAD = 4,     /* pass 2 of one chunk: G staging (the logits     */
+                            /* again, or the kept first-chunk logits)         */
   FLKL_LAUNCH_DW = 5,       /* dW chunk GEMM (fp32 path)                     */
   FLKL_LAUNCH_DX = 6,       /* dX chunk GEMM (fp32 path)                     */
   FLKL_LAUNCH_DB = 7,       /* db column reduction                           */
