@@ -334,9 +334,11 @@ FLKL_API flkl_status flkl_forward_backward_profiled(
  * passes every input and output.
  *
  *  - It allocates nothing and calls no allocating routine.
- *  - Sizes whose flkl_workspace_size() exceeds FLKL_NOALLOC_SCRATCH_BYTES
- *    return FLKL_ERR_TOO_LARGE before any launch (BT=1024, H=4096,
- *    V=128256 with dW needs 98.6 MiB and fits).
+ *  - When flkl_workspace_size() exceeds FLKL_NOALLOC_SCRATCH_BYTES the call
+ *    leaves out the first vocabulary chunk's kept logits and recomputes
+ *    that chunk (the same results; BT=1024, H=4096, V=128256 with dW runs
+ *    so in 119.8 MiB); sizes that need more even then return
+ *    FLKL_ERR_TOO_LARGE before any launch.
  *  - Every call looks up the scratch address on the current device (a
  *    host-side lookup, so a device reset cannot leave a stale address); the
  *    first call on a device also loads the library's device code there, so

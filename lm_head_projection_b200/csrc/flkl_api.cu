@@ -63,7 +63,7 @@ struct Plan {
 };
 
 bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int compute_db,
-               Plan& p) {
+               Plan& p, bool keep_logits = true) {
   (void)compute_dW;
   if (BT < 0 || H < 1 || V < 1) return false;
   if (BT >= (int64_t(1) << 31) || H >= (int64_t(1) << 31) || V >= (int64_t(1) << 31)) return false;
@@ -128,7 +128,7 @@ bool make_plan(int64_t BT, int64_t H, int64_t V, int dtype, int compute_dW, int 
   // of the tile width), so that pass 2 needs no GEMM for them
   const size_t rows32 = size_t(cdiv(BT, 32)) * 32;
   p.zc_cols = 0;
-  if (p.tc && BT > 0)
+  if (p.tc && BT > 0 && keep_logits)
     p.zc_cols = std::min<long long>(
         vc, static_cast<long long>(kLogitCacheBudget / (rows32 * 4)) / p.tile_n * p.tile_n);
   p.off_zc = off;
@@ -998,7 +998,7 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
                                   size_t workspace_bytes, void* stream, Recorder* rec,
                                   const int64_t* target = nullptr,
                                   const int64_t* n_valid_total = nullptr,
-                                  const Phases& ph = Phases{}) {
+                                  const Phases& ph = Phases{}, bool allow_lean = false) {
   // Cross-entropy mode (target set): the teacher is one-hot at target[row],
   // Q is not read and the target doubles as the row mask.
   if (target != nullptr) {
@@ -1035,6 +1035,10 @@ flkl_status forward_backward_impl(const void* X, const void* W, const void* b, c
     return FLKL_ERR_UNSUPPORTED;
   Plan P;
   if (!make_plan(BT, H, V, dtype, compute_dW, compute_db, P)) return FLKL_ERR_INVALID_ARG;
+  // (allow_lean: a workspace that holds all but the first chunk's kept
+  // logits runs with that chunk recomputed; the same results)
+  if (allow_lean && workspace_bytes < P.total)
+    make_plan(BT, H, V, dtype, compute_dW, compute_db, P, false);
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < P.total)
     return FLKL_ERR_WORKSPACE;
@@ -1193,20 +1197,22 @@ flkl_status flkl_forward_backward_noalloc(const void* X, const void* W, const vo
                                           int compute_dW, int compute_db, int accum_fp32,
                                           float* loss, void* dX, void* dW, void* db,
                                           void* stream) {
-  const size_t need = flkl_workspace_size(BT, H, V, dtype, compute_dW, compute_db);
-  if (need == 0) {
+  Plan lean;
+  if (!make_plan(BT, H, V, dtype, compute_dW, compute_db, lean, false)) {
     // invalid sizes or dtype: let the regular validation name the error
     return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
                                  temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
                                  loss, dX, dW, db, nullptr, 0, stream, nullptr);
   }
-  if (need > FLKL_NOALLOC_SCRATCH_BYTES) return FLKL_ERR_TOO_LARGE;
+  // the scratch holds the regular workspace, or at least the one without
+  // the first chunk's kept logits (that chunk is then recomputed)
+  if (lean.total > FLKL_NOALLOC_SCRATCH_BYTES) return FLKL_ERR_TOO_LARGE;
   void* scratch = nullptr;
   if (noalloc_scratch(&scratch) != cudaSuccess) return FLKL_ERR_CUDA;
   return forward_backward_impl(X, W, b, Q, shift_labels, ignore_index, BT, H, V, dtype,
                                temperature, eps, reduction, compute_dW, compute_db, accum_fp32,
                                loss, dX, dW, db, scratch, FLKL_NOALLOC_SCRATCH_BYTES, stream,
-                               nullptr);
+                               nullptr, nullptr, nullptr, Phases{}, true);
 }
 
 flkl_status flkl_forward_backward(const void* X, const void* W, const void* b, const void* Q,

@@ -8,7 +8,9 @@ every device.  These tests call it through the C ABI and check that it gives
 what the workspace entry point gives, within the parity tolerances, on two
 calls in a row (the scratch keeps the previous call's contents, which must
 not leak into the next result), and that sizes beyond the scratch are
-refused before anything runs.  Both entry points run the same deterministic
+refused before anything runs (a size whose regular workspace does not fit
+runs without the first chunk's kept logits, recomputing that chunk, as long
+as the rest fits).  Both entry points run the same deterministic
 kernels on the same bytes, so the results are also compared bitwise; a
 sequence of different plans (a large one, then smaller ones of other dtypes
 and flags, then the large one again) shows that no stale scratch contents
@@ -110,6 +112,24 @@ def test_noalloc_interleaved_plans_give_the_workspace_entry_bytes():
         torch.cuda.synchronize()
         _close(w.dtype, out, ref)
         _same_bytes(out, ref)
+
+
+def test_noalloc_headline_recomputes_the_first_chunk_with_the_same_bytes():
+    """At the headline size the regular workspace (with the first chunk's
+    kept logits) exceeds the scratch; the allocation-free call runs without
+    them, recomputing that chunk, and must give the regular call's bytes."""
+    from lm_head_projection_b200.workloads import WORKLOADS
+
+    w = WORKLOADS["bf16_bt1024_h4096_v128256"]
+    assert pkg.flkl_workspace_size(w.BT, w.H, w.V, 1, 1, 0) > 128 * 2**20
+    dev = torch.device("cuda:0")
+    g = make_inputs(w, device=dev)
+    ref = run_gpu(g)
+    out = {k: (None if ref[k] is None else torch.full_like(ref[k], float("nan")))
+           for k in ("loss", "dX", "dW", "db")}
+    assert _call_noalloc(g, w, out) == 0
+    torch.cuda.synchronize()
+    _same_bytes(out, ref)
 
 
 def test_noalloc_refuses_sizes_beyond_the_scratch():
