@@ -21,7 +21,7 @@
  * section Summary).  The BT x V logits are never written to device memory as
  * a whole: the library computes them tile by tile in two passes (statistics,
  * then the gradient per vocabulary chunk, recomputing the logits) and stages
- * only a bounded BT x Vc block of G (Vc about V/8, rounded up to the tile
+ * only a bounded BT x Vc block of G (Vc about V/6, rounded up to the tile
  * width); on the bf16 path pass 1 keeps the fp32 logits of the first chunk
  * only (at most 256 MiB), from which that chunk's G is formed without a
  * second GEMM.
