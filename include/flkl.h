@@ -199,8 +199,11 @@ FLKL_API flkl_status flkl_selective_logprob_backward(
  *  Xt [BT, Ht], Wt [V, Ht], bt [V] (nullable): teacher hidden states and head,
  *  `dtype` like X; Ht a multiple of 8 (bf16) or 4 (fp32).  0 < beta < 1.
  *  workspace: flkl_jsd_workspace_size bytes (no BT x V buffer: two
- *  staging blocks of one vocabulary chunk).  The probabilities of a chunk are
- *  staged in the input dtype (bf16 on the tensor-core path). */
+ *  staging blocks of one vocabulary chunk and, on the tensor-core path, each
+ *  side's fp32 logits of the first chunk, kept by its statistics pass when
+ *  they fit 256 MiB, so that neither sweep recomputes them).  The
+ *  probabilities of a chunk are staged in the input dtype (bf16 on the
+ *  tensor-core path). */
 FLKL_API size_t flkl_jsd_workspace_size(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype,
                                         int compute_dW, int compute_db);
 FLKL_API flkl_status flkl_jsd_forward_backward(

@@ -616,6 +616,8 @@ struct JsdPlan {
   size_t off_cnt, off_st, off_rows, off_tgt, off_P, off_Q, off_G, off_dx, off_db, total;
   size_t stage;     // bytes of one staging block (BT x Vc elements)
   size_t off_part;  // tensor-core path: [2][n_stat][BT] fp32 partial sums of the loss sweep
+  long long zc_cols;       // tensor-core path: first-chunk logits kept per side (0: none)
+  size_t off_zct, off_zcs; // the teacher's and the student's kept logits
 };
 
 constexpr int kJsdRows = 10;  // fp32 row arrays in the workspace
@@ -667,7 +669,18 @@ bool make_jsd_plan(int64_t BT, int64_t H, int64_t Ht, int64_t V, int dtype, int 
     off += 2 * stage;
     p.off_part = off;
     off += align256(size_t(2) * p.n_stat * BT * 4);
+    // each side's statistics pass keeps the first chunk's logits when the
+    // whole chunk fits the budget, so that neither sweep recomputes that
+    // chunk's logits
+    const size_t zc_bytes = size_t(cdiv(BT, 32)) * 32 * size_t(vc) * 4;
+    p.zc_cols = (BT > 0 && zc_bytes <= kLogitCacheBudget) ? vc : 0;
+    p.off_zct = off;
+    if (p.zc_cols > 0) off += align256(zc_bytes);
+    p.off_zcs = off;
+    if (p.zc_cols > 0) off += align256(zc_bytes);
   } else {
+    p.zc_cols = 0;
+    p.off_zct = p.off_zcs = 0;
     // student and teacher probabilities of one chunk; the gradient block
     // overwrites the student's in place
     p.off_P = off;
@@ -751,13 +764,18 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
   auto chunk_w = [&](long long c) {
     return static_cast<int>(std::min<long long>(P.Vc, V - c * P.Vc));
   };
+  // the first chunk's logits of each side, kept by its statistics pass
+  const bool cached = P.zc_cols > 0;
+  float* zct = reinterpret_cast<float*>(ws + P.off_zct);
+  float* zcs = reinterpret_cast<float*>(ws + P.off_zcs);
   // log-sum-exp of one side: statistics pass (no teacher) + merge
   auto side_lse = [&](const Operand& mA, const Operand& mB, int Hk, const __nv_bfloat16* bias,
-                      float* lse2) -> cudaError_t {
+                      float* lse2, float* zc) -> cudaError_t {
     TcLaunch L = new_launch();
     TcMaps maps{};
     L.stats = EpiStats::Params{nullptr, bias, BT, V, t_scale, 0.f, stats,
-                               static_cast<long long>(P.n_stat) * BT, nt};
+                               static_cast<long long>(P.n_stat) * BT, nt,
+                               cached ? zc : nullptr, static_cast<int>(P.zc_cols)};
     add_problem(L, maps, KIND_STATS, BT, V, Hk, 1, mA, mB);
     cudaError_t e = launch_group(maps, L, st);
     if (e != cudaSuccess) return e;
@@ -768,17 +786,18 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
   };
   // teacher probabilities of chunk c into Qs[c & 1] (the pass-2 epilogue with
   // coefficients 1 and 0 and no target)
+  auto teacher_params = [&](long long c) {
+    return EpiGrad::Params{nullptr, bt,       BT,     V,       chunk_c0(c), ldg, Qs[c & 1],
+                           t_scale, R.lse2_t, R.ones, R.zeros, nullptr,     nt};
+  };
   auto add_teacher = [&](TcLaunch& L, TcMaps& maps, long long c) {
-    const int c0 = chunk_c0(c);
-    L.grad = EpiGrad::Params{nullptr, bt,      BT,      V,       c0,      ldg,     Qs[c & 1],
-                             t_scale, R.lse2_t, R.ones, R.zeros, nullptr, nt};
-    add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), Ht, 1, mXt_k, mWt_k, 0, c0, 0);
+    L.grad = teacher_params(c);
+    add_problem(L, maps, KIND_GRAD, BT, chunk_w(c), Ht, 1, mXt_k, mWt_k, 0, chunk_c0(c), 0);
   };
   // student pass of chunk c, reading Qs[c & 1]
-  auto add_student = [&](TcLaunch& L, TcMaps& maps, long long c, int grad) {
+  auto student_params = [&](long long c, int grad) {
     const int c0 = chunk_c0(c);
-    EpiJsd::Params& j = L.jsd;
-    j = EpiJsd::Params{};
+    EpiJsd::Params j{};
     j.bias = b;
     j.BT = BT;
     j.V = V;
@@ -795,19 +814,42 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
     j.K = R.K;
     j.rowscale = R.rowscale;
     j.dbpart = grad ? dbpart : nullptr;
-    add_problem(L, maps, KIND_JSD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, c0, 0);
+    return j;
+  };
+  auto add_student = [&](TcLaunch& L, TcMaps& maps, long long c, int grad) {
+    L.jsd = student_params(c, grad);
+    add_problem(L, maps, KIND_JSD, BT, chunk_w(c), H, 1, mX_k, mW_k, 0, chunk_c0(c), 0);
   };
   // the teacher pass of chunk 0 alone, then per chunk c: the student pass of
   // chunk c (longer: with the teacher read) and the teacher pass of chunk c+1
+  // (with the kept logits, chunk 0's teacher and student passes are SIMT
+  // kernels on them instead of GEMMs)
+  const int zcols = static_cast<int>(P.zc_cols);
   auto sweep = [&](int grad) -> flkl_status {
-    {
+    if (cached) {
+      const long long warps = cdiv(BT, 32) * (P.zc_cols / 32);
+      k_grad_cached<<<static_cast<unsigned>(cdiv(warps, 8)), 256, 0, st>>>(teacher_params(0),
+                                                                          zct, zcols);
+      FLKL_CUDA(cudaGetLastError());
+    } else {
       TcLaunch L = new_launch();
       TcMaps maps{};
       add_teacher(L, maps, 0);
       FLKL_CUDA(launch_group(maps, L, st));
     }
     for (long long c = 0; c < P.nchunks; ++c) {
-      {
+      if (c == 0 && cached) {
+        const long long warps = cdiv(BT, 32) * (P.zc_cols / TC_EPI_COLS);
+        k_jsd_cached<<<static_cast<unsigned>(cdiv(warps, 8)), 256, 0, st>>>(
+            student_params(0, grad), zcs, zcols);
+        FLKL_CUDA(cudaGetLastError());
+        if (P.nchunks > 1) {
+          TcLaunch L = new_launch();
+          TcMaps maps{};
+          add_teacher(L, maps, 1);
+          FLKL_CUDA(launch_group(maps, L, st));
+        }
+      } else {
         TcLaunch L = new_launch();
         TcMaps maps{};
         add_student(L, maps, c, grad);
@@ -834,8 +876,8 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
     return FLKL_OK;
   };
 
-  FLKL_CUDA(side_lse(mXt_k, mWt_k, Ht, bt, R.lse2_t));
-  FLKL_CUDA(side_lse(mX_k, mW_k, H, b, R.lse2_s));
+  FLKL_CUDA(side_lse(mXt_k, mWt_k, Ht, bt, R.lse2_t, zct));
+  FLKL_CUDA(side_lse(mX_k, mW_k, H, b, R.lse2_s, zcs));
   k_jsd_init_rows<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
       labels, BT, ignore_index, ctl, R.rowscale, R.K, R.L);
   FLKL_CUDA(cudaGetLastError());
@@ -848,8 +890,11 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
   s = sweep(1);
   if (s != FLKL_OK) return s;
   if (compute_db) {
+    // the 32-row groups that hold rows (k_jsd_cached writes no partials for
+    // the all-padding groups of the last row tile; the GEMM epilogues write
+    // zeros there)
     k_db_reduce<<<static_cast<unsigned>(cdiv(V, 256)), 256, 0, st>>>(
-        dbpart, static_cast<int>(P.db_groups), V, db, accum_fp32);
+        dbpart, static_cast<int>(cdiv(BT, 32)), V, db, accum_fp32);
     FLKL_CUDA(cudaGetLastError());
   }
   return FLKL_OK;

@@ -442,6 +442,65 @@ struct EpiJsd {
       prefetch_l2(q + 64);
     }
   }
+  // The 32 columns [gcol0, gcol0 + 32) of one row (lane = row of a 32-row
+  // group) from the student logits z (the accumulator, before the bias) and
+  // the staged teacher probabilities q: loss mode adds p ln(p/m) and
+  // q ln(q/m) into kp and kq; gradient mode writes the row's 32 gradients
+  // (bf16) at column col0 of G and, with db, the group's column sums.  Shared
+  // by the epilogue and k_jsd_cached, which therefore give the same bits.
+  __device__ __forceinline__ static void cols32(const Params& p, float (&z)[32],
+                                                const float (&q)[32], int row, bool rv,
+                                                int rgroup, int col0, int gcol0, float lse2,
+                                                float gk, float gs, float& kp, float& kq,
+                                                int lane) {
+    const float LN2 = 0.693147180559945309f;
+    const float beta = p.beta, omb = 1.f - p.beta;
+    if (p.bias != nullptr) {  // warp-uniform
+      float bv[32];
+      load_bias32(p.bias, gcol0, p.V, bv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) z[i] += bv[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const bool ok = (gcol0 + i) < p.V;
+      // p rounded to bf16 like the staged teacher q, so that a teacher equal
+      // to the student gives p == q exactly (divergence and gradient 0)
+      const float pv =
+          ok ? __bfloat162float(__float2bfloat16_rn(exp2f(__fmaf_rn(z[i], p.t_scale, -lse2))))
+             : 0.f;
+      const float qv = ok ? q[i] : 0.f;
+      const float mv = __fmaf_rn(beta, pv, omb * qv);
+      const float lm = __log2f(mv);
+      // p ln(p/m) and q ln(q/m), 0 when the probability is 0
+      const float lp = pv > 0.f ? (__log2f(pv) - lm) * LN2 : 0.f;
+      if (!p.grad) {
+        kp = __fmaf_rn(pv, lp, kp);
+        if (qv > 0.f) kq = __fmaf_rn(qv, (__log2f(qv) - lm) * LN2, kq);
+      } else {
+        z[i] = pv > 0.f ? gs * pv * (lp - gk) : 0.f;
+      }
+    }
+    if (p.grad) {
+      if (rv) {
+        uint4* dst = reinterpret_cast<uint4*>(p.G + static_cast<size_t>(row) * p.ldg + col0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 u;
+          u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
+          u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
+          u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
+          u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
+          dst[j] = u;
+        }
+      }
+      if (p.dbpart != nullptr) {
+        const float colsum = warp_transpose_sum32(z, lane);
+        const int gc = gcol0 + lane;
+        if (gc < p.V) p.dbpart[static_cast<size_t>(rgroup) * p.V + gc] = colsum;
+      }
+    }
+  }
   __device__ __forceinline__ static void run(const Params& p, uint32_t taddr, int row0, int n0,
                                              int quad, int lane) {
     const int row = row0 + quad * 32 + lane;
@@ -449,10 +508,8 @@ struct EpiJsd {
     if (p.c0 + n0 >= p.V) return;  // warp-uniform
     const __nv_bfloat16* qrow = p.Qs + static_cast<size_t>(rv ? row : 0) * p.ldg;
     const float lse2 = rv ? p.lse2[row] : 0.f;
-    const float LN2 = 0.693147180559945309f;
-    const float beta = p.beta, omb = 1.f - p.beta;
     const float gk = (p.grad && rv) ? p.K[row] : 0.f;
-    const float gs = (p.grad && rv) ? p.rowscale[row] * beta : 0.f;
+    const float gs = (p.grad && rv) ? p.rowscale[row] * p.beta : 0.f;
     float kp = 0.f, kq = 0.f;
     uint4 qa[4], qb[4];
     load_chunk32_rw(qrow, rv, n0, p.ldg, qa);
@@ -461,65 +518,66 @@ struct EpiJsd {
       const int col0 = n0 + c * 32;
       const int gcol0 = p.c0 + col0;
       if (gcol0 >= p.V) break;  // warp-uniform
-      float q[32], bv[32], z[32];
+      float q[32], z[32];
       if (c + 1 < TC_EPI_COLS / 32) load_chunk32_rw(qrow, rv, col0 + 32, p.ldg, qb);
 #pragma unroll
       for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
       tmem_ld32(taddr + c * 32, z);
-      if (p.bias != nullptr) {  // warp-uniform
-        load_bias32(p.bias, gcol0, p.V, bv);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) z[i] += bv[i];
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool ok = (gcol0 + i) < p.V;
-        // p rounded to bf16 like the staged teacher q, so that a teacher equal
-        // to the student gives p == q exactly (divergence and gradient 0)
-        const float pv = ok ? __bfloat162float(__float2bfloat16_rn(exp2f(z[i] * p.t_scale - lse2)))
-                            : 0.f;
-        const float qv = ok ? q[i] : 0.f;
-        const float mv = beta * pv + omb * qv;
-        const float lm = __log2f(mv);
-        // p ln(p/m) and q ln(q/m), 0 when the probability is 0
-        const float lp = pv > 0.f ? (__log2f(pv) - lm) * LN2 : 0.f;
-        if (!p.grad) {
-          kp = fmaf(pv, lp, kp);
-          kq += qv > 0.f ? qv * ((__log2f(qv) - lm) * LN2) : 0.f;
-        } else {
-          z[i] = pv > 0.f ? gs * pv * (lp - gk) : 0.f;
-        }
-      }
-      if (p.grad) {
-        if (rv) {
-          uint4* dst = reinterpret_cast<uint4*>(p.G + static_cast<size_t>(row) * p.ldg + col0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 u;
-            u.x = pack_bf16x2(z[8 * j + 0], z[8 * j + 1]);
-            u.y = pack_bf16x2(z[8 * j + 2], z[8 * j + 3]);
-            u.z = pack_bf16x2(z[8 * j + 4], z[8 * j + 5]);
-            u.w = pack_bf16x2(z[8 * j + 6], z[8 * j + 7]);
-            dst[j] = u;
-          }
-        }
-        if (p.dbpart != nullptr) {
-          const float colsum = warp_transpose_sum32(z, lane);
-          const int gc = gcol0 + lane;
-          if (gc < p.V)
-            p.dbpart[static_cast<size_t>(row0 / 32 + quad) * p.V + gc] = colsum;
-        }
-      }
+      cols32(p, z, q, row, rv, row0 / 32 + quad, col0, gcol0, lse2, gk, gs, kp, kq, lane);
 #pragma unroll
       for (int j = 0; j < 4; ++j) qa[j] = qb[j];
     }
     if (!p.grad && rv) {
       const size_t o = static_cast<size_t>((p.c0 + n0) / TC_EPI_COLS) * p.BT + row;
       p.part[o] = kp;
-      p.part[o + p.part_plane] = beta * kp + omb * kq;
+      p.part[o + p.part_plane] = __fmaf_rn(p.beta, kp, (1.f - p.beta) * kq);
     }
   }
 };
+
+// The student pass of the first vocabulary chunk from the logits its
+// statistics pass kept (EpiStats::Params::zc, same layout as for
+// k_grad_cached): one warp per 32 rows x 128 columns (a statistics group),
+// lane = row, the four 32-column blocks in order, EpiJsd::cols32 as in the
+// epilogue; loss mode writes the group's partial sums, gradient mode the
+// gradient block over the staged teacher block.  8 warps per block.
+__global__ void __launch_bounds__(256) k_jsd_cached(const EpiJsd::Params p,
+                                                    const float* __restrict__ zc, int zc_cols) {
+  const int lane = threadIdx.x & 31;
+  const int ngrp = zc_cols / TC_EPI_COLS;
+  const long long w = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (w >= static_cast<long long>((p.BT + 31) >> 5) * ngrp) return;  // warp-uniform
+  const int rg = static_cast<int>(w / ngrp), n0 = static_cast<int>(w % ngrp) * TC_EPI_COLS;
+  if (p.c0 + n0 >= p.V) return;  // warp-uniform
+  const int row = rg * 32 + lane;
+  const bool rv = row < p.BT;
+  const __nv_bfloat16* qrow = p.Qs + static_cast<size_t>(rv ? row : 0) * p.ldg;
+  const float lse2 = rv ? p.lse2[row] : 0.f;
+  const float gk = (p.grad && rv) ? p.K[row] : 0.f;
+  const float gs = (p.grad && rv) ? p.rowscale[row] * p.beta : 0.f;
+  float kp = 0.f, kq = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < TC_EPI_COLS / 32; ++c) {
+    const int col0 = n0 + c * 32;
+    const int gcol0 = p.c0 + col0;
+    if (gcol0 >= p.V) break;  // warp-uniform
+    uint4 qa[4];
+    load_chunk32_rw(qrow, rv, col0, p.ldg, qa);
+    float q[32], z[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack8_bf16(qa[j], q + 8 * j);
+    const float* src =
+        zc + (static_cast<size_t>(rg) * (zc_cols >> 5) + (col0 >> 5)) * 1024 + lane;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) z[i] = rv ? src[i * 32] : 0.f;
+    EpiJsd::cols32(p, z, q, row, rv, rg, col0, gcol0, lse2, gk, gs, kp, kq, lane);
+  }
+  if (!p.grad && rv) {
+    const size_t o = static_cast<size_t>((p.c0 + n0) / TC_EPI_COLS) * p.BT + row;
+    p.part[o] = kp;
+    p.part[o + p.part_plane] = __fmaf_rn(p.beta, kp, (1.f - p.beta) * kq);
+  }
+}
 
 // dW rows of one chunk: out[c0 + m][n] = acc, fp32 or bf16.
 // The store epilogues read the accumulator in the 16-lane fragment layout

@@ -247,4 +247,4 @@ def test_jsd_entry_checks_its_arguments():
     assert jsd(compute_db=1, db=P) == INVALID  # db needs a bias
     assert jsd(workspace_bytes=100) == WORKSPACE
     need = pkg.flkl_jsd_workspace_size(1024, 4096, 4096, 128256, 1, 1, 0)
-    assert 0 < need < 1024 * 128256 * 2 // 2   # no BT x V buffer
+    assert 0 < need < 1024 * 128256 * 2   # below one BT x V bf16 array
