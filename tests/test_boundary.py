@@ -248,3 +248,18 @@ def test_jsd_entry_checks_its_arguments():
     assert jsd(workspace_bytes=100) == WORKSPACE
     need = pkg.flkl_jsd_workspace_size(1024, 4096, 4096, 128256, 1, 1, 0)
     assert 0 < need < 1024 * 128256 * 2   # below one BT x V bf16 array
+
+
+def test_launch_kind_names_follow_the_header_enum():
+    """The binding's names of the profiled launch kinds are the header's
+    flkl_launch_kind values, in order."""
+    import os
+    import re
+
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "flkl.h")).read()
+    body = hdr[hdr.index("typedef enum {\n  FLKL_LAUNCH_PREPARE"):hdr.index("} flkl_launch_kind;")]
+    vals = {int(v): n for n, v in re.findall(r"FLKL_LAUNCH_(\w+)\s*=\s*(\d+)", body)}
+    assert sorted(vals) == list(range(len(vals)))
+    names = [vals[i].lower() for i in range(len(vals))]
+    assert [n.replace("_", "") for n in names] == [k.replace("_", "").lower()
+                                                   for k in pkg.LAUNCH_KINDS]
