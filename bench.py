@@ -1014,6 +1014,7 @@ def run_jsd(args):
     ms = e0.elapsed_time(e1) / args.steps
     peaks, peak_src = load_peaks()
     # counted: teacher and student logits, dX and dW; executed: 8 such GEMMs
+    # less the first vocabulary chunk's four (formed from the kept logits)
     counted = 2.0 * w.BT * w.V * w.H * 4
     achieved = counted / (ms * 1e-3) / 1e12
     from oracle import jsd_forward_backward as oracle_jsd
@@ -1038,7 +1039,8 @@ def run_jsd(args):
                      "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "traffic": None,
                      "scope": "whole call; counted = teacher + student logits, dX, dW "
-                              "(8 GEMMs of that size run); burst peak",
+                              "(8 GEMMs of that size run, less the first vocabulary "
+                              "chunk's four chunk-sized ones); burst peak",
                      "peak_source": peak_src},
         "cpu_baseline": {"value": round(rows / t_cpu, 2), "unit": "tokens/s",
                          "cores": host_threads(), "kind": "oracle",

@@ -883,7 +883,7 @@ flkl_status run_jsd_tc(const JsdPlan& P, const __nv_bfloat16* X, const __nv_bflo
   FLKL_CUDA(cudaGetLastError());
   flkl_status s = sweep(0);
   if (s != FLKL_OK) return s;
-  k_jsd_sum_parts<<<static_cast<unsigned>(cdiv(BT, 256)), 256, 0, st>>>(
+  k_jsd_sum_parts<<<static_cast<unsigned>(cdiv(BT, 32)), 32 * kJsdSumWarps, 0, st>>>(
       part, static_cast<int>(P.n_stat), BT, R.rowscale, R.K, R.scrL);
   k_loss<<<1, 1024, 0, st>>>(R.scrL, BT, ctl, loss);
   FLKL_CUDA(cudaGetLastError());

@@ -82,22 +82,40 @@ __global__ void __launch_bounds__(256) k_jsd_rows(const T* __restrict__ P, const
   }
 }
 
-// Tensor-core path: K[r] and the row loss from the loss sweep's partial sums
-// part[0][g][r] (of p ln(p/m)) and part[1][g][r] (of the row loss), summed
-// over the column groups g in order; dropped rows get 0.
-__global__ void k_jsd_sum_parts(const float* __restrict__ part, int n_groups, int BT,
-                                const float* __restrict__ rowscale, float* __restrict__ K,
-                                float* __restrict__ rowloss) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= BT) return;
+// K_r = sum over the column groups of the loss sweep's partial sums of
+// KL(P_r||M_r), and the row's loss (0 on dropped rows), in a fixed order: one
+// block of 32 warps per 32 rows, warp w adding groups w, w + 32, ... (loads
+// coalesced over the 32 rows), then warp 0 adding the 32 warp sums in warp
+// order.
+constexpr int kJsdSumWarps = 32;
+__global__ void __launch_bounds__(32 * kJsdSumWarps)
+    k_jsd_sum_parts(const float* __restrict__ part, int n_groups, int BT,
+                    const float* __restrict__ rowscale, float* __restrict__ K,
+                    float* __restrict__ rowloss) {
+  __shared__ float sk[kJsdSumWarps][33], sl[kJsdSumWarps][33];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int r = blockIdx.x * 32 + lane;
   const size_t plane = static_cast<size_t>(n_groups) * BT;
   float k = 0.f, l = 0.f;
-  for (int g = 0; g < n_groups; ++g) {
-    k += part[static_cast<size_t>(g) * BT + r];
-    l += part[plane + static_cast<size_t>(g) * BT + r];
+  if (r < BT) {
+#pragma unroll 4
+    for (int g = w; g < n_groups; g += kJsdSumWarps) {
+      k += part[static_cast<size_t>(g) * BT + r];
+      l += part[plane + static_cast<size_t>(g) * BT + r];
+    }
   }
-  K[r] = k;
-  rowloss[r] = rowscale[r] != 0.f ? l : 0.f;
+  sk[w][lane] = k;
+  sl[w][lane] = l;
+  __syncthreads();
+  if (w == 0 && r < BT) {
+    float kk = sk[0][lane], ll = sl[0][lane];
+    for (int i = 1; i < kJsdSumWarps; ++i) {
+      kk += sk[i][lane];
+      ll += sl[i][lane];
+    }
+    K[r] = kk;
+    rowloss[r] = rowscale[r] != 0.f ? ll : 0.f;
+  }
 }
 
 // Row losses of kept rows (dropped rows 0) for the fixed-order reduction.
